@@ -1,0 +1,394 @@
+#!/usr/bin/env python
+"""Benchmark of the fine-grained FP8 hot path on B200.
+
+One step = one pass of the whole path over one batch of the dense workload
+(A bf16 [4096, 7168] ~N(0,1) with 0.1% x100 outliers, W bf16 [7168, 7168] ~N(0,0.006),
+power-of-two scales, bf16 output):
+    quant_act_1x128(A) -> quant_weight_128x128(W) -> gemm_blockscaled(qA, sA, qW, sW)
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+
+Prints one JSON line (rank 0).  ``value`` is GEMM FLOPs of all ranks / device time of
+the whole step (quantization included), max over ranks; per-kernel event times give the
+live roofline of the dominant kernel.  L2 is flushed (512 MB write) between steps,
+outside the per-step events.  ``--impl reference`` times the CPU oracle (the reference
+arm of this project) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "FP8 block-scaled GEMM TFLOP/s and % of FP8 tensor peak; quant GB/s and % of HBM"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FP8_PER_BF16 = 2.0   # nominal dense fp8 : bf16 tensor throughput ratio
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return (float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]),
+                "measured")
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS * 0.88, "fallback"
+
+
+# ------------------------------------------------------------------------------ clocks (NVML)
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons every ~20 ms in a thread while active."""
+
+    REASONS = {0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x4: "sw_power_cap", 0x1: "gpu_idle",
+               0x2: "applications_clocks_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._nv is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": float(statistics.median(self.samples)) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------ distributed
+
+def dist_init(args):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl != "reference":
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------ GPU arm
+
+def dev_bf16(bits):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def run_gpu(args, rank, world):
+    import torch
+    import fp8_fine_grained_weight_b200 as fq
+
+    w = workloads.ALL[args.workload]()
+    assert not w.experts, "the bench times the dense path"
+    M, N, K = w.M, w.N, w.K
+    G = K // 128
+    a_bits, b_bits = w.gen_a(), w.gen_b()
+    A, W = dev_bf16(a_bits), dev_bf16(b_bits)
+    qA = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    sA = torch.empty((G, M), dtype=torch.float32, device="cuda")
+    qW = torch.empty((N, K), dtype=torch.uint8, device="cuda")
+    sW = torch.empty((N // 128, G), dtype=torch.float32, device="cuda")
+    out_dtype = torch.float32 if w.out_fp32 else torch.bfloat16
+    C = torch.empty((M, N), dtype=out_dtype, device="cuda")
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        fq.quant_act_1x128(A, w.pow2_a, out=(qA, sA))
+        if ev is not None:
+            ev[1].record(stream)
+        fq.quant_weight_128x128(W, w.pow2_b, out=(qW, sW))
+        if ev is not None:
+            ev[2].record(stream)
+        fq.gemm_blockscaled(qA, sA, qW, sW, out=C)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    err = fq.device_error()
+    if err:
+        raise RuntimeError(f"device error word {err:#x} after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for i in range(args.steps):
+            flush.zero_()          # L2 flush, outside the step's events
+            step(evs[i])
+        torch.cuda.synchronize()
+    barrier(world)
+    t_act = [e[0].elapsed_time(e[1]) for e in evs]
+    t_w = [e[1].elapsed_time(e[2]) for e in evs]
+    t_gemm = [e[2].elapsed_time(e[3]) for e in evs]
+    t_step = [e[0].elapsed_time(e[3]) for e in evs]
+    ms_step = max_over_ranks(sum(t_step) / len(t_step), world)
+    ms_act = sum(t_act) / len(t_act)
+    ms_w = sum(t_w) / len(t_w)
+    ms_gemm = sum(t_gemm) / len(t_gemm)
+    if fq.device_error():
+        raise RuntimeError("device error word set after the timed region")
+
+    hbm, bf16_burst, bf16_sust, peak_src = peaks()
+    fp8_peak = bf16_burst * FP8_PER_BF16
+    flops = w.gemm_flops
+    gemm_tflops = flops / (ms_gemm * 1e-3) / 1e12
+    act_bytes = M * K * 2 + M * K + M * G * 4
+    w_bytes = N * K * 2 + N * K + (N // 128) * G * 4
+    value = world * flops / (ms_step * 1e-3) / 1e12
+
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "gemm_dense_traffic.json")
+    if os.path.exists(tp):
+        try:
+            tj = json.load(open(tp))
+            if tj.get("workload") == w.name and tj.get("kernel_rev") == kernel_rev():
+                traffic = tj.get("dram_bytes_per_launch")
+        except Exception:
+            traffic = None
+
+    res = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 x e4m3 -> f32 accumulate, bf16 out", "data": "synthetic",
+        "config": {"workload": w.name, "M": M, "N": N, "K": K, "pow2_scales": True,
+                   "out": "bf16" if not w.out_fp32 else "fp32",
+                   "parallelism": f"replicas x{world} (dense: each GPU its own 4096-token batch)",
+                   "l2": "512 MB flush write between steps, outside the per-step events"},
+        "kernels_ms": {"quant_act_1x128": round(ms_act, 5), "quant_weight_128x128": round(ms_w, 5),
+                       "gemm_blockscaled": round(ms_gemm, 5)},
+        "gemm_tflops": round(gemm_tflops, 1),
+        "gemm_frac_of_fp8_peak": round(gemm_tflops / fp8_peak, 4),
+        "gemm_frac_of_fp8_spec_4500": round(gemm_tflops / 4500.0, 4),
+        "quant_act_gbs": round(act_bytes / (ms_act * 1e-3) / 1e9, 1),
+        "quant_act_frac_hbm": round(act_bytes / (ms_act * 1e-3) / 1e9 / hbm, 4),
+        "quant_weight_gbs": round(w_bytes / (ms_w * 1e-3) / 1e9, 1),
+        "quant_weight_frac_hbm": round(w_bytes / (ms_w * 1e-3) / 1e9 / hbm, 4),
+        "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 1),
+                     "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+                     "frac": round(gemm_tflops / fp8_peak, 4), "traffic": traffic,
+                     "kernel": "gemm_blockscaled",
+                     "peak_source": f"{peak_src} bf16 burst {bf16_burst} x {FP8_PER_BF16} (fp8:bf16)"},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk.summary(),
+    }
+
+    # ---- end to end through the public API with host buffers
+    e2e_steps = max(3, min(args.steps, args.e2e_steps))
+    A_h = torch.from_numpy(a_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    W_h = torch.from_numpy(b_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    C_h = torch.empty((M, N), dtype=out_dtype).pin_memory()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def e2e_step():
+        A.copy_(A_h, non_blocking=True)
+        W.copy_(W_h, non_blocking=True)
+        step()
+        C_h.copy_(C, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(ev0.elapsed_time(ev1) / e2e_steps, world)
+    res["e2e"] = {"value": round(world * flops / (ms_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                  "h2d_bytes_per_step": int(A_h.numel() * 2 + W_h.numel() * 2),
+                  "d2h_bytes_per_step": int(C_h.numel() * C_h.element_size()),
+                  "ms_per_step": round(ms_e2e, 4), "steps": e2e_steps}
+
+    # ---- parity spot check of this run's output against the oracle (rank 0, 4 rows)
+    if rank == 0 and not args.no_check:
+        res["spot_check"] = spot_check(w, a_bits, b_bits, C)
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w, a_bits, b_bits, budget_s=args.cpu_budget)
+    return res
+
+
+def kernel_rev() -> str:
+    """Short hash of the kernel sources, to tie stored ncu counters to the code they measured."""
+    import hashlib
+    h = hashlib.sha1()
+    for f in ("ptx.cuh", "quant.cuh", "gemm.cuh", "fp8q.cu"):
+        h.update(open(os.path.join(ROOT, "fp8_fine_grained_weight_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:12]
+
+
+def spot_check(w, a_bits, b_bits, C):
+    import oracle
+    rows = np.array([0, 1, w.M // 2, w.M - 1])
+    qa, sa = oracle.quant_act_1x128(a_bits[rows], w.pow2_a)
+    qb, sb = oracle.quant_weight_128x128(b_bits, w.pow2_b)
+    C_ref, T = oracle.gemm_blockscaled_ref(qa, sa, qb, sb)
+    import torch
+    Ch = C[torch.from_numpy(rows).cuda()].float().cpu().numpy().astype(np.float64)
+    ok, fb = oracle.check_bf16(Ch, C_ref, T) if not w.out_fp32 else (oracle.check_fp32(Ch, C_ref, T), None)
+    return {"rows": rows.tolist(), "within_band": bool(ok.all()), "entries": int(ok.size)}
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+
+def cpu_baseline(w, a_bits, b_bits, budget_s: float = 20.0):
+    """The oracle, as it stands, on the host cores: W quantized in full once, then A rows in
+    chunks (1x128 quantization + FP64 dequantize + dgemm) until the budget is spent; the
+    per-step time is extrapolated to all M rows."""
+    import oracle
+    cores = os.cpu_count()
+    t0 = time.perf_counter()
+    qb, sb = oracle.quant_weight_128x128(b_bits, w.pow2_b)
+    Bd = oracle.dequant_blocks(qb, sb)
+    t_w = time.perf_counter() - t0
+    rows_done, t_rows, chunk = 0, 0.0, 64
+    while t_rows < budget_s and rows_done < w.M:
+        t1 = time.perf_counter()
+        r = slice(rows_done, min(w.M, rows_done + chunk))
+        qa, sa = oracle.quant_act_1x128(a_bits[r], w.pow2_a)
+        Ad = oracle.dequant_rows_groupmajor(qa, sa)
+        _ = Ad @ Bd.T
+        t_rows += time.perf_counter() - t1
+        rows_done = r.stop
+    t_step = t_w + t_rows * (w.M / rows_done)
+    return {"value": round(w.gemm_flops / t_step / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"full W quantization ({t_w:.2f} s) + {rows_done} of {w.M} A rows "
+                      f"(quantize, FP64 dequantize, dgemm: {t_rows:.2f} s), per-step time "
+                      f"extrapolated to all rows; numpy BLAS and OpenMP threads = host cores"}
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle on a bounded sample per step (8 rows x 128 columns)."""
+    import oracle
+    w = workloads.ALL[args.workload]()
+    rng = np.random.default_rng(0)
+    a_bits = workloads.normal_bf16(rng, (8, w.K), w.a_std, w.a_outliers)
+    b_bits = workloads.normal_bf16(rng, (128, w.K), w.b_std)
+    flops = 2.0 * 8 * 128 * w.K
+
+    def step():
+        qa, sa = oracle.quant_act_1x128(a_bits, w.pow2_a)
+        qb, sb = oracle.quant_weight_128x128(b_bits, w.pow2_b)
+        oracle.gemm_blockscaled_ref(qa, sa, qb, sb)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    v = round(flops / dt / 1e12, 6)
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(dt * 1e3, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64 (oracle)", "data": "synthetic",
+            "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": os.cpu_count(),
+                             "kind": "oracle",
+                             "sample": f"per step: 8 rows x 128 columns x K={w.K} of the workload "
+                                       f"(1x128 + 128x128 quantization, FP64 GEMM)"},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="dense", choices=["tiny", "dense", "wgrad"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-check", action="store_true")
+    args = ap.parse_args()
+
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    rank, world, _ = dist_init(args)
+    res = run_gpu(args, rank, world)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,238 @@
+"""fp8q: fine-grained FP8 (E4M3) quantization and block-scaled FP8 GEMM on B200 (sm_100a).
+
+A thin ctypes binding over ``libfp8q.so`` (the C ABI in ``include/fp8q.h``).  Every
+step of the computation runs in the library's CUDA kernels; this module only checks
+tensor dtypes/devices, allocates outputs with PyTorch and passes raw device pointers
+and the current CUDA stream.  There is no CPU fallback: if the library is missing or
+a call fails, an exception is raised.
+
+Layouts (see include/fp8q.h):
+  activation scales  group-major fp32 [K/128, ld]   (scale of row m, group g at [g, m])
+  weight scales      fp32 [N/128, K/128]
+  E4M3 tensors       torch.uint8 (view as torch.float8_e4m3fn if wanted)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp8q.so")
+
+OUT_BF16, OUT_FP32 = 0, 1
+BSCALE_BLOCK, BSCALE_ROW = 0, 1
+
+STATUS = {0: "FP8Q_OK", 1: "FP8Q_ERR_NULL", 2: "FP8Q_ERR_SHAPE", 3: "FP8Q_ERR_ALIGN",
+          4: "FP8Q_ERR_UNSUPPORTED", 5: "FP8Q_ERR_CUDA", 6: "FP8Q_ERR_TIMEOUT"}
+
+# name -> (restype, argtypes); mirrors include/fp8q.h
+_i64, _i32, _vp, _f = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_float
+SIGNATURES = {
+    "fp8q_quant_act_1x128": (_i32, [_vp, _i64, _i64, _i64, _vp, _i64, _vp, _i64, _i32, _vp]),
+    "fp8q_quant_weight_128x128": (_i32, [_vp, _i64, _i64, _i64, _vp, _i64, _vp, _i32, _vp]),
+    "fp8q_quant_rowwise": (_i32, [_vp, _i64, _i64, _i64, _vp, _i64, _vp, _i32, _vp]),
+    "fp8_gemm_blockscaled": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _i32, _vp, _i32,
+                                    _i64, _i64, _i64, _i64, _i64, _i64, _vp]),
+    "fp8_gemm_grouped": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _i32, _vp, _i32,
+                                _i64, _i64, _i64, _vp]),
+    "fp8_gemm_nopromo": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _vp]),
+    "fp8q_get_device_error": (_i32, [_vp]),
+    "fp8q_status_string": (ctypes.c_char_p, [_i32]),
+    "fp8q_abi_version": (_i32, []),
+}
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+class Fp8qError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS.get(status & 0xFF, status)} "
+                         f"({lib().fp8q_status_string(status).decode()}), site {status >> 8}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library.  Raises if ``libfp8q.so`` has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m fp8_fine_grained_weight_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _call(name: str, *args) -> None:
+    st = getattr(lib(), name)(*args)
+    if st != 0:
+        raise Fp8qError(name, st)
+
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _need(t: torch.Tensor, dtype, name: str, ndim: Optional[int] = None) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    if t.dim() and t.stride(-1) != 1:
+        raise ValueError(f"{name} must be contiguous in its last dimension")
+
+
+def _u8(t: torch.Tensor) -> torch.Tensor:
+    return t.view(torch.uint8) if t.dtype == torch.float8_e4m3fn else t
+
+
+# --------------------------------------------------------------------------------------
+# quantization
+# --------------------------------------------------------------------------------------
+
+def quant_act_1x128(x: torch.Tensor, pow2: bool = False, ld_scale: Optional[int] = None,
+                    out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None):
+    """1x128 activation tiles: x bf16 [M, K] -> (q uint8 [M, K], s fp32 [K/128, ld_scale])."""
+    _need(x, torch.bfloat16, "x", 2)
+    M, K = x.shape
+    ld = M if ld_scale is None else int(ld_scale)
+    if out is None:
+        q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+        s = torch.empty((K // 128 if K % 128 == 0 else 0, ld), dtype=torch.float32, device=x.device)
+    else:
+        q, s = out
+    _call("fp8q_quant_act_1x128", x.data_ptr(), M, K, x.stride(0), q.data_ptr(), q.stride(0),
+          s.data_ptr(), ld, int(bool(pow2)), _stream(x))
+    return q, s
+
+
+def quant_weight_128x128(w: torch.Tensor, pow2: bool = False,
+                         out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None):
+    """128x128 weight blocks: w bf16 [N, K] (or [E, N, K]) -> (q uint8, s fp32 [.., N/128, K/128])."""
+    _need(w, torch.bfloat16, "w")
+    if w.dim() not in (2, 3):
+        raise ValueError("w must be [N, K] or [E, N, K]")
+    if not w.is_contiguous():
+        raise ValueError("w must be contiguous")
+    K = w.shape[-1]
+    N_all = w.numel() // K if K else 0
+    if out is None:
+        q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+        s = torch.empty((*w.shape[:-2], w.shape[-2] // 128, K // 128), dtype=torch.float32,
+                        device=w.device)
+    else:
+        q, s = out
+    _call("fp8q_quant_weight_128x128", w.data_ptr(), N_all, K, K, q.data_ptr(), K, s.data_ptr(),
+          int(bool(pow2)), _stream(w))
+    return q, s
+
+
+def quant_rowwise(x: torch.Tensor, pow2: bool = False):
+    """One scale per row over all of K: x bf16 [M, K] -> (q uint8 [M, K], s fp32 [M])."""
+    _need(x, torch.bfloat16, "x", 2)
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    s = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _call("fp8q_quant_rowwise", x.data_ptr(), M, K, x.stride(0), q.data_ptr(), q.stride(0),
+          s.data_ptr(), int(bool(pow2)), _stream(x))
+    return q, s
+
+
+# --------------------------------------------------------------------------------------
+# GEMM
+# --------------------------------------------------------------------------------------
+
+def _out_code(out_dtype) -> int:
+    if out_dtype == torch.bfloat16:
+        return OUT_BF16
+    if out_dtype == torch.float32:
+        return OUT_FP32
+    raise TypeError("out_dtype must be torch.bfloat16 or torch.float32")
+
+
+def gemm_blockscaled(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor,
+                     out_dtype=torch.bfloat16, b_rowwise: bool = False,
+                     out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """C = A B^T with per-128-K promotion.
+
+    qa uint8 [M, K]; sa fp32 [K/128, >= M]; qb uint8 [N, K];
+    sb fp32 [N/128, K/128] (128x128 blocks) or, with ``b_rowwise``, [K/128, >= N].
+    """
+    qa, qb = _u8(qa), _u8(qb)
+    _need(qa, torch.uint8, "qa", 2)
+    _need(qb, torch.uint8, "qb", 2)
+    _need(sa, torch.float32, "sa", 2)
+    _need(sb, torch.float32, "sb", 2)
+    M, K = qa.shape
+    N = qb.shape[0]
+    if qb.shape[1] != K:
+        raise ValueError("qa and qb disagree on K")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=qa.device)
+    _call("fp8_gemm_blockscaled", qa.data_ptr(), sa.data_ptr(), sa.stride(0), qb.data_ptr(),
+          sb.data_ptr(), sb.stride(0) if b_rowwise else 0,
+          BSCALE_ROW if b_rowwise else BSCALE_BLOCK, out.data_ptr(), _out_code(out.dtype),
+          M, N, K, qa.stride(0), qb.stride(0), out.stride(0), _stream(qa))
+    return out
+
+
+def gemm_grouped(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor,
+                 m_offsets: torch.Tensor, out_dtype=torch.bfloat16,
+                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """MoE grouped GEMM: rows m_offsets[e]..m_offsets[e+1] of A times W[e]^T.
+
+    qa uint8 [sumM, K]; sa fp32 [K/128, >= sumM]; qw uint8 [E, N, K]; sw fp32 [E, N/128, K/128];
+    m_offsets int32 [E + 1] on the device (read by the kernel, no host sync).
+    """
+    qa, qw = _u8(qa), _u8(qw)
+    _need(qa, torch.uint8, "qa", 2)
+    _need(qw, torch.uint8, "qw", 3)
+    _need(sa, torch.float32, "sa", 2)
+    _need(sw, torch.float32, "sw", 3)
+    _need(m_offsets, torch.int32, "m_offsets", 1)
+    if not (qa.is_contiguous() and qw.is_contiguous() and sw.is_contiguous()):
+        raise ValueError("qa, qw and sw must be contiguous")
+    M, K = qa.shape
+    E, N, _ = qw.shape
+    if m_offsets.numel() != E + 1:
+        raise ValueError("m_offsets must have E + 1 entries")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=qa.device)
+    _call("fp8_gemm_grouped", qa.data_ptr(), sa.data_ptr(), sa.stride(0), qw.data_ptr(),
+          sw.data_ptr(), out.data_ptr(), _out_code(out.dtype), m_offsets.data_ptr(), E, M, N, K,
+          _stream(qa))
+    return out
+
+
+def gemm_nopromo(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor,
+                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Accumulation-study variant: one accumulator over all of K, 1xK scales sa [M], sb [N]; fp32 C."""
+    qa, qb = _u8(qa), _u8(qb)
+    _need(qa, torch.uint8, "qa", 2)
+    _need(qb, torch.uint8, "qb", 2)
+    _need(sa, torch.float32, "sa", 1)
+    _need(sb, torch.float32, "sb", 1)
+    M, K = qa.shape
+    N = qb.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=qa.device)
+    _call("fp8_gemm_nopromo", qa.data_ptr(), sa.data_ptr(), qb.data_ptr(), sb.data_ptr(),
+          out.data_ptr(), M, N, K, qa.stride(0), qb.stride(0), out.stride(0), _stream(qa))
+    return out
+
+
+def device_error(device=None) -> int:
+    """Read and clear the library's device error word (synchronizes the current stream)."""
+    return int(lib().fp8q_get_device_error(torch.cuda.current_stream(device).cuda_stream))
+
+
+def status_string(status: int) -> str:
+    return lib().fp8q_status_string(int(status)).decode()

@@ -1,0 +1,280 @@
+// libfp8q.so: the C ABI declared in include/fp8q.h.
+//
+// Host side: argument validation (before any launch), TMA tensor-map encoding
+// (cuTensorMapEncodeTiled through the runtime's driver entry point, so the library
+// needs no -lcuda), kernel attribute setup and launches on the caller's stream.
+// All device code lives in quant.cuh and gemm.cuh (one translation unit).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "../../include/fp8q.h"
+#include "gemm.cuh"
+#include "quant.cuh"
+
+namespace {
+
+using fp8q::GemmArgs;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  return n;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2D K-major E4M3 operand: [rows, K] with a row stride of `ld` bytes; box = 128 bytes of K
+// by `box_rows` rows, 128-byte swizzle (the canonical layout the MMA descriptors expect).
+int encode_operand(CUtensorMap* tm, const void* base, uint64_t K, uint64_t rows, uint64_t ld,
+                   uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return FP8Q_ERR_CUDA;
+  cuuint64_t dims[2] = {K, rows};
+  cuuint64_t strides[1] = {ld};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+template <bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16>
+int launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& args, int grid,
+                cudaStream_t stream) {
+  auto kern = fp8q::gemm_fp8_blockscaled_kernel<PROMOTE, ROW_B, GROUPED, OUT_BF16>;
+  static std::atomic<bool> configured[64];  // per instantiation, per device
+  const int smem = static_cast<int>(fp8q::SmemLayout::bytes);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8Q_ERR_CUDA;
+  if (!configured[dev].load(std::memory_order_acquire)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return FP8Q_ERR_CUDA;
+    configured[dev].store(true, std::memory_order_release);
+  }
+  kern<<<grid, fp8q::kGemmThreads, smem, stream>>>(tmA, tmB, args);
+  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+int check_gemm_common(const uint8_t* A, const uint8_t* B, const void* C, int out_dtype,
+                             int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
+                             int64_t ldc) {
+  if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_SHAPE;
+  if (out_dtype != FP8Q_OUT_BF16 && out_dtype != FP8Q_OUT_FP32) return FP8Q_ERR_UNSUPPORTED;
+  if (!A || !B || !C) return FP8Q_ERR_NULL;
+  if (K == 0 || K % 128 != 0 || N == 0 || N % 128 != 0) return FP8Q_ERR_SHAPE;
+  if (lda < K || ldb < K || ldc < N) return FP8Q_ERR_SHAPE;
+  const int64_t esz = out_dtype == FP8Q_OUT_BF16 ? 2 : 4;
+  if (lda % 16 != 0 || ldb % 16 != 0 || (ldc * esz) % 16 != 0) return FP8Q_ERR_ALIGN;
+  if (!aligned(A, 16) || !aligned(B, 16) || !aligned(C, 16)) return FP8Q_ERR_ALIGN;
+  if (K / 128 > 0x7FFFFF || M > 0x7FFFFFFF || N > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
+  return FP8Q_OK;
+}
+
+template <bool PROMOTE, bool GROUPED>
+int dispatch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
+                         bool row_b, bool bf16, int grid, cudaStream_t st) {
+  if (row_b) {
+    return bf16 ? launch_gemm<PROMOTE, true, GROUPED, true>(tmA, tmB, a, grid, st)
+                : launch_gemm<PROMOTE, true, GROUPED, false>(tmA, tmB, a, grid, st);
+  }
+  return bf16 ? launch_gemm<PROMOTE, false, GROUPED, true>(tmA, tmB, a, grid, st)
+              : launch_gemm<PROMOTE, false, GROUPED, false>(tmA, tmB, a, grid, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fp8q_abi_version(void) { return 1; }
+
+const char* fp8q_status_string(int status) {
+  switch (status & 0xFF) {
+    case FP8Q_OK: return "ok";
+    case FP8Q_ERR_NULL: return "null pointer argument";
+    case FP8Q_ERR_SHAPE: return "invalid shape or leading dimension";
+    case FP8Q_ERR_ALIGN: return "pointer or leading dimension misaligned";
+    case FP8Q_ERR_UNSUPPORTED: return "unsupported mode, dtype or device";
+    case FP8Q_ERR_CUDA: return "CUDA call failed";
+    case FP8Q_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int fp8q_get_device_error(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned int h = 0;
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, fp8q::g_device_error) != cudaSuccess) return FP8Q_ERR_CUDA;
+  if (cudaMemcpyAsync(&h, addr, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return FP8Q_ERR_CUDA;
+  if (cudaMemsetAsync(addr, 0, sizeof(h), s) != cudaSuccess) return FP8Q_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FP8Q_ERR_CUDA;
+  return static_cast<int>(h);
+}
+
+int fp8q_quant_act_1x128(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, int64_t ldq,
+                         float* scales, int64_t ld_scale, int pow2_scale, void* stream) {
+  if (M < 0 || K < 0) return FP8Q_ERR_SHAPE;
+  if (M == 0 || K == 0) return FP8Q_OK;
+  if (!x || !q || !scales) return FP8Q_ERR_NULL;
+  if (K % 128 != 0 || ldx < K || ldq < K || ld_scale < M) return FP8Q_ERR_SHAPE;
+  if (ldx % 8 != 0 || ldq % 8 != 0 || !aligned(x, 16) || !aligned(q, 8) || !aligned(scales, 4))
+    return FP8Q_ERR_ALIGN;
+  const int64_t G = K / 128;
+  if (G > 65535) return FP8Q_ERR_SHAPE;
+  dim3 grid(static_cast<unsigned>((M + fp8q::kActRowsPerBlock - 1) / fp8q::kActRowsPerBlock),
+            static_cast<unsigned>(G));
+  auto st = static_cast<cudaStream_t>(stream);
+  const auto* xs = static_cast<const uint16_t*>(x);
+  if (pow2_scale)
+    fp8q::quant_act_1x128_kernel<true><<<grid, 256, 0, st>>>(xs, M, ldx, q, ldq, scales, ld_scale);
+  else
+    fp8q::quant_act_1x128_kernel<false><<<grid, 256, 0, st>>>(xs, M, ldx, q, ldq, scales, ld_scale);
+  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+int fp8q_quant_weight_128x128(const void* w, int64_t N, int64_t K, int64_t ldw, uint8_t* q,
+                              int64_t ldq, float* scales, int pow2_scale, void* stream) {
+  if (N < 0 || K < 0) return FP8Q_ERR_SHAPE;
+  if (N == 0 || K == 0) return FP8Q_OK;
+  if (!w || !q || !scales) return FP8Q_ERR_NULL;
+  if (N % 128 != 0 || K % 128 != 0 || ldw < K || ldq < K) return FP8Q_ERR_SHAPE;
+  if (ldw % 8 != 0 || ldq % 8 != 0 || !aligned(w, 16) || !aligned(q, 8) || !aligned(scales, 4))
+    return FP8Q_ERR_ALIGN;
+  const int64_t G = K / 128, NB = N / 128;
+  if (NB > 65535 || G > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
+  dim3 grid(static_cast<unsigned>(G), static_cast<unsigned>(NB));
+  auto st = static_cast<cudaStream_t>(stream);
+  const auto* ws = static_cast<const uint16_t*>(w);
+  if (pow2_scale)
+    fp8q::quant_weight_128x128_kernel<true><<<grid, 256, 0, st>>>(ws, ldw, q, ldq, scales, G);
+  else
+    fp8q::quant_weight_128x128_kernel<false><<<grid, 256, 0, st>>>(ws, ldw, q, ldq, scales, G);
+  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+int fp8q_quant_rowwise(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, int64_t ldq,
+                       float* scales, int pow2_scale, void* stream) {
+  if (M < 0 || K < 0) return FP8Q_ERR_SHAPE;
+  if (M == 0 || K == 0) return FP8Q_OK;
+  if (!x || !q || !scales) return FP8Q_ERR_NULL;
+  if (K % 128 != 0 || ldx < K || ldq < K) return FP8Q_ERR_SHAPE;
+  if (ldx % 8 != 0 || ldq % 8 != 0 || !aligned(x, 16) || !aligned(q, 8) || !aligned(scales, 4))
+    return FP8Q_ERR_ALIGN;
+  if (M > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
+  auto st = static_cast<cudaStream_t>(stream);
+  const auto* xs = static_cast<const uint16_t*>(x);
+  if (pow2_scale)
+    fp8q::quant_rowwise_kernel<true><<<static_cast<unsigned>(M), 256, 0, st>>>(xs, K, ldx, q, ldq, scales);
+  else
+    fp8q::quant_rowwise_kernel<false><<<static_cast<unsigned>(M), 256, 0, st>>>(xs, K, ldx, q, ldq, scales);
+  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+int fp8_gemm_blockscaled(const uint8_t* A, const float* sA, int64_t ld_sa, const uint8_t* B,
+                         const float* sB, int64_t ld_sb, int b_scale_mode, void* C, int out_dtype,
+                         int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
+                         void* stream) {
+  if (M == 0 && N >= 0 && K >= 0) return FP8Q_OK;
+  int st = check_gemm_common(A, B, C, out_dtype, M, N, K, lda, ldb, ldc);
+  if (st != FP8Q_OK) return st;
+  if (!sA || !sB) return FP8Q_ERR_NULL;
+  if (b_scale_mode != FP8Q_BSCALE_BLOCK128x128 && b_scale_mode != FP8Q_BSCALE_ROW1x128)
+    return FP8Q_ERR_UNSUPPORTED;
+  if (ld_sa < M) return FP8Q_ERR_SHAPE;
+  if (b_scale_mode == FP8Q_BSCALE_ROW1x128 && ld_sb < N) return FP8Q_ERR_SHAPE;
+  if (!aligned(sA, 4) || !aligned(sB, 4)) return FP8Q_ERR_ALIGN;
+  const int sms = device_sm_count();
+  if (sms <= 0) return FP8Q_ERR_CUDA;
+
+  CUtensorMap tmA, tmB;
+  if ((st = encode_operand(&tmA, A, K, M, lda, fp8q::kBM)) != FP8Q_OK) return st;
+  if ((st = encode_operand(&tmB, B, K, N, ldb, fp8q::kBN)) != FP8Q_OK) return st;
+  GemmArgs a{};
+  a.sA = sA; a.ld_sa = ld_sa; a.sB = sB; a.ld_sb = ld_sb; a.C = C; a.ldc = ldc;
+  a.M = M; a.N = N; a.G = static_cast<int>(K / 128); a.m_offsets = nullptr; a.num_experts = 0;
+  const int64_t tiles = ((M + fp8q::kBM - 1) / fp8q::kBM) * ((N + fp8q::kBN - 1) / fp8q::kBN);
+  if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  return dispatch_gemm<true, false>(tmA, tmB, a, b_scale_mode == FP8Q_BSCALE_ROW1x128,
+                                    out_dtype == FP8Q_OUT_BF16, grid, static_cast<cudaStream_t>(stream));
+}
+
+int fp8_gemm_grouped(const uint8_t* A, const float* sA, int64_t ld_sa, const uint8_t* W,
+                     const float* sW, void* C, int out_dtype, const int32_t* m_offsets,
+                     int num_groups, int64_t max_sum_M, int64_t N, int64_t K, void* stream) {
+  if (max_sum_M < 0 || N < 0 || K < 0) return FP8Q_ERR_SHAPE;
+  if (num_groups < 1 || num_groups > fp8q::kMaxGroups) return FP8Q_ERR_UNSUPPORTED;
+  if (max_sum_M == 0) return FP8Q_OK;
+  int st = check_gemm_common(A, W, C, out_dtype, max_sum_M, N, K, K, K, N);
+  if (st != FP8Q_OK) return st;
+  if (!sA || !sW || !m_offsets) return FP8Q_ERR_NULL;
+  if (ld_sa < max_sum_M) return FP8Q_ERR_SHAPE;
+  if (!aligned(sA, 4) || !aligned(sW, 4) || !aligned(m_offsets, 4)) return FP8Q_ERR_ALIGN;
+  if (static_cast<int64_t>(num_groups) * N > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
+  const int sms = device_sm_count();
+  if (sms <= 0) return FP8Q_ERR_CUDA;
+
+  CUtensorMap tmA, tmB;
+  if ((st = encode_operand(&tmA, A, K, max_sum_M, K, fp8q::kBM)) != FP8Q_OK) return st;
+  if ((st = encode_operand(&tmB, W, K, static_cast<uint64_t>(num_groups) * N, K, fp8q::kBN)) != FP8Q_OK)
+    return st;
+  GemmArgs a{};
+  a.sA = sA; a.ld_sa = ld_sa; a.sB = sW; a.ld_sb = 0; a.C = C; a.ldc = N;
+  a.M = max_sum_M; a.N = N; a.G = static_cast<int>(K / 128);
+  a.m_offsets = m_offsets; a.num_experts = num_groups;
+  // Upper bound on tiles (every group may add one partial m-tile) sizes the persistent grid.
+  const int64_t nt = (N + fp8q::kBN - 1) / fp8q::kBN;
+  const int64_t bound = ((max_sum_M + fp8q::kBM - 1) / fp8q::kBM + num_groups) * nt;
+  if (bound > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
+  const int grid = static_cast<int>(bound < sms ? bound : sms);
+  return dispatch_gemm<true, true>(tmA, tmB, a, false, out_dtype == FP8Q_OUT_BF16, grid,
+                                   static_cast<cudaStream_t>(stream));
+}
+
+int fp8_gemm_nopromo(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB, float* C,
+                     int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
+                     void* stream) {
+  if (M == 0 && N >= 0 && K >= 0) return FP8Q_OK;
+  int st = check_gemm_common(A, B, C, FP8Q_OUT_FP32, M, N, K, lda, ldb, ldc);
+  if (st != FP8Q_OK) return st;
+  if (!sA || !sB) return FP8Q_ERR_NULL;
+  if (!aligned(sA, 4) || !aligned(sB, 4)) return FP8Q_ERR_ALIGN;
+  const int sms = device_sm_count();
+  if (sms <= 0) return FP8Q_ERR_CUDA;
+  CUtensorMap tmA, tmB;
+  if ((st = encode_operand(&tmA, A, K, M, lda, fp8q::kBM)) != FP8Q_OK) return st;
+  if ((st = encode_operand(&tmB, B, K, N, ldb, fp8q::kBN)) != FP8Q_OK) return st;
+  GemmArgs a{};
+  a.sA = sA; a.ld_sa = 0; a.sB = sB; a.ld_sb = 0; a.C = C; a.ldc = ldc;
+  a.M = M; a.N = N; a.G = static_cast<int>(K / 128); a.m_offsets = nullptr; a.num_experts = 0;
+  const int64_t tiles = ((M + fp8q::kBM - 1) / fp8q::kBM) * ((N + fp8q::kBN - 1) / fp8q::kBN);
+  if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  return launch_gemm<false, false, false, false>(tmA, tmB, a, grid, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,125 @@
+"""Host-only checks of the C ABI: the library loads, exports every function that
+include/fp8q.h declares, and rejects bad arguments before any launch.
+
+No call here reaches a kernel launch or any CUDA call (validation returns first), so
+these run on a machine without a GPU.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8q.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from fp8_fine_grained_weight_b200 import build
+    build.build()
+    import fp8_fine_grained_weight_b200 as fq
+    return fq.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b((?:fp8q|fp8)_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_expected_entry_points():
+    names = declared_functions()
+    for want in ("fp8q_quant_act_1x128", "fp8q_quant_weight_128x128", "fp8_gemm_blockscaled",
+                 "fp8_gemm_grouped", "fp8q_get_device_error", "fp8q_status_string"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    import fp8_fine_grained_weight_b200 as fq
+    for name in declared_functions():
+        assert hasattr(L, name), name
+        assert name in fq.SIGNATURES, f"binding lacks {name}"
+
+
+def test_status_strings_and_version(L):
+    assert L.fp8q_abi_version() == 1
+    assert L.fp8q_status_string(0) == b"ok"
+    assert b"timed out" in L.fp8q_status_string(6)
+    assert L.fp8q_status_string(6 | (4 << 8)) == L.fp8q_status_string(6)
+    assert L.fp8q_status_string(99) == b"unknown status"
+
+
+NULL = None
+P16 = 0x10000          # a fake, 16-byte aligned "device" address: never dereferenced
+P_MIS = 0x10004        # misaligned by 4
+
+
+def test_quant_act_validation(L):
+    f = L.fp8q_quant_act_1x128
+    assert f(P16, 0, 128, 128, P16, 128, P16, 0, 0, NULL) == 0          # empty: no-op
+    assert f(P16, -1, 128, 128, P16, 128, P16, 1, 0, NULL) == 2
+    assert f(NULL, 4, 128, 128, P16, 128, P16, 4, 0, NULL) == 1
+    assert f(P16, 4, 100, 128, P16, 128, P16, 4, 0, NULL) == 2          # K % 128
+    assert f(P16, 4, 128, 64, P16, 128, P16, 4, 0, NULL) == 2           # ldx < K
+    assert f(P16, 4, 128, 128, P16, 128, P16, 3, 0, NULL) == 2          # ld_scale < M
+    assert f(P_MIS, 4, 128, 128, P16, 128, P16, 4, 0, NULL) == 3        # x misaligned
+    assert f(P16, 4, 128, 132, P16, 128, P16, 4, 0, NULL) == 3          # ldx % 8
+
+
+def test_quant_weight_validation(L):
+    f = L.fp8q_quant_weight_128x128
+    assert f(P16, 0, 128, 128, P16, 128, P16, 0, NULL) == 0
+    assert f(P16, 100, 128, 128, P16, 128, P16, 0, NULL) == 2           # N % 128
+    assert f(P16, 128, 128, 128, NULL, 128, P16, 0, NULL) == 1
+    assert f(P_MIS, 128, 128, 128, P16, 128, P16, 0, NULL) == 3
+
+
+def test_gemm_validation(L):
+    f = L.fp8_gemm_blockscaled
+    ok_args = dict(A=P16, sA=P16, ld_sa=256, B=P16, sB=P16, ld_sb=0, mode=0, C=P16, out=0,
+                   M=256, N=256, K=256, lda=256, ldb=256, ldc=256)
+
+    def call(**kw):
+        a = dict(ok_args, **kw)
+        return f(a["A"], a["sA"], a["ld_sa"], a["B"], a["sB"], a["ld_sb"], a["mode"], a["C"],
+                 a["out"], a["M"], a["N"], a["K"], a["lda"], a["ldb"], a["ldc"], NULL)
+
+    assert call(M=0) == 0                      # empty problem: no-op
+    assert call(A=NULL) == 1
+    assert call(sB=NULL) == 1
+    assert call(K=200, lda=256, ldb=256) == 2  # K % 128
+    assert call(N=200) == 2                    # N % 128
+    assert call(M=-5) == 2
+    assert call(lda=128) == 2                  # lda < K
+    assert call(ld_sa=100) == 2                # ld_sa < M
+    assert call(mode=1, ld_sb=100) == 2        # ROW mode needs ld_sb >= N
+    assert call(mode=7) == 4
+    assert call(out=3) == 4
+    assert call(A=P_MIS) == 3
+    assert call(lda=264) == 3                  # not a multiple of 16
+    assert call(ldc=260, out=0) == 3           # 520 B row pitch is not a multiple of 16
+
+
+def test_grouped_validation(L):
+    f = L.fp8_gemm_grouped
+    assert f(P16, P16, 64, P16, P16, P16, 0, P16, 0, 64, 256, 256, NULL) == 4      # no groups
+    assert f(P16, P16, 64, P16, P16, P16, 0, P16, 2000, 64, 256, 256, NULL) == 4   # too many
+    assert f(P16, P16, 64, P16, P16, P16, 0, P16, 4, 0, 256, 256, NULL) == 0       # empty
+    assert f(P16, P16, 64, P16, P16, P16, 0, NULL, 4, 64, 256, 256, NULL) == 1
+    assert f(P16, P16, 32, P16, P16, P16, 0, P16, 4, 64, 256, 256, NULL) == 2      # ld_sa
+    assert f(P16, P16, 64, P16, P16, P16, 0, P16, 4, 64, 256, 200, NULL) == 2      # K
+
+
+def test_nopromo_validation(L):
+    f = L.fp8_gemm_nopromo
+    assert f(P16, P16, P16, P16, P16, 0, 256, 256, 256, 256, 256, NULL) == 0
+    assert f(P16, NULL, P16, P16, P16, 4, 256, 256, 256, 256, 256, NULL) == 1
+    assert f(P16, P16, P16, P16, P16, 4, 250, 256, 256, 256, 256, NULL) == 2
+
+
+def test_binding_refuses_cpu_tensors():
+    torch = pytest.importorskip("torch")
+    import fp8_fine_grained_weight_b200 as fq
+    with pytest.raises(TypeError):
+        fq.quant_act_1x128(torch.zeros(4, 128, dtype=torch.bfloat16))

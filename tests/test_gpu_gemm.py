@@ -1,0 +1,248 @@
+"""GPU parity of the block-scaled FP8 GEMMs against the FP64 oracle, through the C ABI.
+
+Acceptance: fp32 output |C - C_ref| <= 2e-5 sum_k|a~ b~| + 1e-30; bf16 output within
+1 bf16 ulp of C_ref (cancellation fallback: the bf16 rounding of a value inside the
+fp32 band); the unit-scale integer case bit-exact.  Inputs are quantized by each side
+on its own (the GPU's codes are first checked bit-exact against the oracle's).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from tests._helpers import (assert_bytes_equal, assert_gemm_close, host, rel_err_stats, to_dev,
+                            to_dev_bf16)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fq():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import fp8_fine_grained_weight_b200 as fq
+    fq.lib()
+    return fq
+
+
+def _dense_case(fq, a_bits, b_bits, pow2_a, pow2_b, out_fp32, b_rowwise=False, rows=None,
+                name="dense"):
+    """Quantize on both sides, check the codes, run the GEMM, compare (sampled) rows."""
+    import torch
+    a, b = to_dev_bf16(a_bits), to_dev_bf16(b_bits)
+    qa, sa = fq.quant_act_1x128(a, pow2_a)
+    if b_rowwise:
+        qb, sb = fq.quant_act_1x128(b, pow2_b)
+    else:
+        qb, sb = fq.quant_weight_128x128(b, pow2_b)
+    out_dtype = torch.float32 if out_fp32 else torch.bfloat16
+    C = fq.gemm_blockscaled(qa, sa, qb, sb, out_dtype=out_dtype, b_rowwise=b_rowwise)
+    torch.cuda.synchronize()
+    assert fq.device_error() == 0
+
+    rows = np.arange(a_bits.shape[0]) if rows is None else np.asarray(rows)
+    qa_ref, sa_ref = oracle.quant_act_1x128(a_bits[rows], pow2_a)
+    if b_rowwise:
+        qb_ref, sb_ref = oracle.quant_act_1x128(b_bits, pow2_b)
+    else:
+        qb_ref, sb_ref = oracle.quant_weight_128x128(b_bits, pow2_b)
+    assert_bytes_equal(name + ".qa", host(qa)[rows], qa_ref)
+    assert_bytes_equal(name + ".qb", host(qb), qb_ref)
+    C_ref, T = oracle.gemm_blockscaled_ref(qa_ref, sa_ref, qb_ref, sb_ref, b_rowwise)
+    Ch = host(C)[rows]
+    fb = assert_gemm_close(name, Ch, C_ref, T, bf16=not out_fp32)
+    return Ch, C_ref, T, fb
+
+
+def test_tiny_fp32(fq):
+    w = workloads.tiny()
+    C, C_ref, T, _ = _dense_case(fq, w.gen_a(), w.gen_b(), False, False, True, name="tiny")
+    mx, med = rel_err_stats(C, C_ref, T)
+    assert mx <= 2e-5
+
+
+def test_tiny_unit_scale_integers_exact(fq):
+    """qA, qB small E4M3 integers, unit scales: every partial sum is an integer below 2^14,
+    so the result must equal the integer product exactly."""
+    import torch
+    rng = workloads.rng_for(1, 9)
+    qa, ia = workloads.small_int_e4m3_codes(rng, (128, 512))
+    qb, ib = workloads.small_int_e4m3_codes(rng, (256, 512))
+    sa = np.ones((4, 128), np.float32)
+    sb = np.ones((2, 4), np.float32)
+    C = fq.gemm_blockscaled(to_dev(qa), to_dev(sa), to_dev(qb), to_dev(sb), out_dtype=torch.float32)
+    want = (ia @ ib.T).astype(np.float32)
+    assert_bytes_equal("unit-scale C", host(C), want)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 128, 128), (129, 256, 128), (200, 384, 640),
+                                   (257, 512, 256), (64, 128, 1024), (300, 1280, 384)])
+@pytest.mark.parametrize("out_fp32", [True, False])
+def test_ragged_shapes(fq, M, N, K, out_fp32):
+    rng = np.random.default_rng(M + 3 * N + 7 * K)
+    a = workloads.normal_bf16(rng, (M, K), 1.0, 0.01)
+    b = workloads.normal_bf16(rng, (N, K), 0.02)
+    _dense_case(fq, a, b, False, False, out_fp32, name=f"ragged {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("M,N,K", [(77, 256, 512), (128, 384, 256)])
+def test_rowwise_b_scales(fq, M, N, K):
+    rng = np.random.default_rng(M * N)
+    a = workloads.normal_bf16(rng, (M, K), 1e-3)
+    b = workloads.normal_bf16(rng, (N, K), 1.0)
+    _dense_case(fq, a, b, False, False, True, b_rowwise=True, name="row-b")
+
+
+def test_linearity_per_group_on_gpu(fq):
+    """Doubling the A scales of group g adds the group-g term (within the fp32 band)."""
+    import torch
+    rng = np.random.default_rng(21)
+    a = workloads.normal_bf16(rng, (128, 512), 1.0)
+    b = workloads.normal_bf16(rng, (256, 512), 0.02)
+    qa, sa = fq.quant_act_1x128(to_dev_bf16(a), False)
+    qb, sb = fq.quant_weight_128x128(to_dev_bf16(b), False)
+    C0 = host(fq.gemm_blockscaled(qa, sa, qb, sb, out_dtype=torch.float32)).astype(np.float64)
+    qa_ref, sa_ref = oracle.quant_act_1x128(a, False)
+    qb_ref, sb_ref = oracle.quant_weight_128x128(b, False)
+    for g in range(4):
+        sa2 = sa.clone()
+        sa2[g] *= 2
+        C2 = host(fq.gemm_blockscaled(qa, sa2, qb, sb, out_dtype=torch.float32)).astype(np.float64)
+        qg = qa_ref.copy()
+        mask = np.ones(512, bool)
+        mask[g * 128:(g + 1) * 128] = False
+        qg[:, mask] = 0
+        Cg, Tg = oracle.gemm_blockscaled_ref(qg, sa_ref, qb_ref, sb_ref)
+        _, T = oracle.gemm_blockscaled_ref(qa_ref, sa_ref, qb_ref, sb_ref)
+        assert np.all(np.abs((C2 - C0) - Cg) <= 2e-5 * (2 * T + Tg) + 1e-30)
+
+
+def test_dense_full_size_sampled_rows(fq):
+    """The dense workload at full size, in the bench's launch configuration; 96 sampled
+    rows (spanning every M tile and the last row) compared with the oracle."""
+    w = workloads.dense()
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([rng.choice(w.M, 94, replace=False), [0, w.M - 1]]))
+    _, _, _, fb = _dense_case(fq, w.gen_a(), w.gen_b(), True, True, False, rows=rows,
+                              name="dense full")
+
+
+def test_wgrad_full_size_sampled_rows(fq):
+    w = workloads.wgrad()
+    rng = np.random.default_rng(1)
+    rows = np.unique(np.concatenate([rng.choice(w.M, 30, replace=False), [w.M - 1]]))
+    C, C_ref, T, _ = _dense_case(fq, w.gen_a(), w.gen_b(), False, False, True, b_rowwise=True,
+                                 rows=rows, name="wgrad full")
+
+
+# ------------------------------------------------------------------------------------ grouped
+
+def _grouped_case(fq, counts, N, K, pow2_a, out_fp32, a_std=1.0, b_std=0.006, rows=None,
+                  seed=0, bits=None, name="grouped"):
+    import torch
+    counts = np.asarray(counts, dtype=np.int64)
+    E = counts.size
+    off = workloads.offsets_from_counts(counts)
+    M = int(off[-1])
+    if bits is None:
+        rng = np.random.default_rng(seed)
+        a_bits = workloads.normal_bf16(rng, (max(M, 1), K), a_std, 0.001)
+        w_bits = workloads.normal_bf16(rng, (E, N, K), b_std)
+    else:
+        a_bits, w_bits = bits
+    qa, sa = fq.quant_act_1x128(to_dev_bf16(a_bits), pow2_a)
+    qw, sw = fq.quant_weight_128x128(to_dev_bf16(w_bits), False)
+    out_dtype = torch.float32 if out_fp32 else torch.bfloat16
+    C = torch.full((max(M, 1), N), float("nan"), dtype=out_dtype, device="cuda")
+    fq.gemm_grouped(qa, sa, qw, sw, to_dev(off), out_dtype=out_dtype, out=C)
+    torch.cuda.synchronize()
+    assert fq.device_error() == 0
+    if M == 0:
+        return
+    rows = np.arange(M) if rows is None else np.asarray(rows)
+    qa_ref, sa_ref = oracle.quant_act_1x128(a_bits[rows], pow2_a)
+    assert_bytes_equal(name + ".qa", host(qa)[rows], qa_ref)
+    # experts touched by the sampled rows
+    expert = np.searchsorted(off, rows, side="right") - 1
+    qw_h, sw_h = host(qw), host(sw)
+    for e in np.unique(expert):
+        q_ref, s_ref = oracle.quant_weight_128x128(w_bits[e], False)
+        assert_bytes_equal(f"{name}.qw[{e}]", qw_h[e], q_ref)
+        assert_bytes_equal(f"{name}.sw[{e}]", sw_h[e], s_ref)
+    # oracle over the sampled rows: sA columns re-indexed to the sampled rows
+    qa_full = np.zeros((M, K), np.uint8)
+    qa_full[rows] = qa_ref
+    sa_full = np.zeros((K // 128, M), np.float32)
+    sa_full[:, rows] = sa_ref
+    qw_ref = np.stack([oracle.quant_weight_128x128(w_bits[e], False)[0] if e in expert else
+                       np.zeros((N, K), np.uint8) for e in range(E)])
+    sw_ref = np.stack([oracle.quant_weight_128x128(w_bits[e], False)[1] if e in expert else
+                       np.ones((N // 128, K // 128), np.float32) for e in range(E)])
+    C_ref, T = oracle.gemm_grouped_ref(qa_full, sa_full, qw_ref, sw_ref, off, rows=rows)
+    assert_gemm_close(name, host(C)[rows], C_ref, T, bf16=not out_fp32)
+
+
+@pytest.mark.parametrize("out_fp32", [True, False])
+def test_grouped_small_with_empty_groups(fq, out_fp32):
+    _grouped_case(fq, [0, 5, 130, 1, 0, 77, 256, 0], 256, 384, False, out_fp32, seed=1)
+
+
+def test_grouped_unwritten_rows_untouched(fq):
+    """Rows past the last offset (allocation slack) are not written."""
+    import torch
+    rng = np.random.default_rng(2)
+    counts = np.array([3, 0, 40])
+    off = workloads.offsets_from_counts(counts)
+    a = workloads.normal_bf16(rng, (64, 256), 1.0)
+    w = workloads.normal_bf16(rng, (3, 128, 256), 0.02)
+    qa, sa = fq.quant_act_1x128(to_dev_bf16(a), False)
+    qw, sw = fq.quant_weight_128x128(to_dev_bf16(w), False)
+    C = torch.full((64, 128), 7.0, dtype=torch.float32, device="cuda")
+    fq.gemm_grouped(qa, sa, qw, sw, to_dev(off), out_dtype=torch.float32, out=C)
+    assert np.all(host(C)[43:] == 7.0)
+
+
+def test_grouped_all_empty(fq):
+    _grouped_case(fq, [0, 0, 0], 128, 256, False, True, seed=3)
+
+
+def test_grouped_decode_full_size(fq):
+    """64 experts, M_e ~ U{1..256}, W [7168, 2048]; every 9th row compared."""
+    w = workloads.decode()
+    rows = np.arange(0, w.M, 9)
+    _grouped_case(fq, w.counts, w.N, w.K, True, False, rows=rows, bits=(w.gen_a(), w.gen_b()),
+                  name="decode full")
+
+
+def test_grouped_prefill_full_size(fq):
+    """32 experts, Zipf routing (sum M ~ 87K), W [4096, 7168]; sampled rows of 4 experts."""
+    w = workloads.prefill()
+    off = w.offsets
+    rng = np.random.default_rng(4)
+    rows = []
+    for e in (0, 1, 17, 31):
+        lo, hi = int(off[e]), int(off[e + 1])
+        rows += list(rng.choice(np.arange(lo, hi), 12, replace=False)) + [hi - 1]
+    _grouped_case(fq, w.counts, w.N, w.K, False, False, rows=np.array(sorted(set(rows))),
+                  bits=(w.gen_a(), w.gen_b()), name="prefill full")
+
+
+# ------------------------------------------------------------------------------ no promotion
+
+def test_nopromo_matches_oracle_on_rowwise_codes(fq):
+    """One accumulator over all of K: compared with FP64 on the same 1xK codes."""
+    import torch
+    rng = np.random.default_rng(6)
+    a = workloads.normal_bf16(rng, (200, 2048), 1e-3)
+    b = workloads.normal_bf16(rng, (256, 2048), 1.0)
+    qa, sa = fq.quant_rowwise(to_dev_bf16(a))
+    qb, sb = fq.quant_rowwise(to_dev_bf16(b))
+    C = fq.gemm_nopromo(qa, sa, qb, sb)
+    qa_r, sa_r = oracle.quant_rowwise(a)
+    qb_r, sb_r = oracle.quant_rowwise(b)
+    assert_bytes_equal("nopromo.qa", host(qa), qa_r)
+    C_ref, T = oracle.gemm_ref(oracle.dequant_rowwise(qa_r, sa_r), oracle.dequant_rowwise(qb_r, sb_r))
+    # no acceptance band is claimed for this variant; it must still be a close FP32 result
+    mx, _ = rel_err_stats(host(C), C_ref, T)
+    assert mx < 1e-3
