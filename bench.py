@@ -10,8 +10,8 @@ power-of-two scales, bf16 output):
 
 Prints one JSON line (rank 0).  ``value`` is GEMM FLOPs of all ranks / device time of
 the whole step (quantization included), max over ranks; per-kernel event times give the
-live roofline of the dominant kernel.  L2 is flushed (512 MB write) between steps,
-outside the per-step events.  ``--impl reference`` times the CPU oracle (the reference
+live roofline of the dominant kernel.  L2 is flushed between steps (a 512 MB write,
+then a read of it so no dirty lines remain), outside the per-step events.  ``--impl reference`` times the CPU oracle (the reference
 arm of this project) on a bounded sample of the same workload.
 """
 from __future__ import annotations
@@ -170,8 +170,14 @@ def run_gpu(args, rank, world):
         if ev is not None:
             ev[3].record(stream)
 
-    for _ in range(max(args.warmup, 3)):
+    def flush_l2():
+        # write a buffer 4x the L2, then read it back: the inputs are evicted and the
+        # L2 holds no dirty lines that the first timed kernel would have to write back
         flush.zero_()
+        flush.view(torch.int64).sum()
+
+    for _ in range(max(args.warmup, 3)):
+        flush_l2()
         step()
     torch.cuda.synchronize()
     err = fq.device_error()
@@ -183,7 +189,7 @@ def run_gpu(args, rank, world):
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
         for i in range(args.steps):
-            flush.zero_()          # L2 flush, outside the step's events
+            flush_l2()             # outside the step's events
             step(evs[i])
         torch.cuda.synchronize()
     barrier(world)
@@ -224,7 +230,7 @@ def run_gpu(args, rank, world):
         "config": {"workload": w.name, "M": M, "N": N, "K": K, "pow2_scales": True,
                    "out": "bf16" if not w.out_fp32 else "fp32",
                    "parallelism": f"replicas x{world} (dense: each GPU its own 4096-token batch)",
-                   "l2": "512 MB flush write between steps, outside the per-step events"},
+                   "l2": "flush between steps (512 MB write, then read back), outside the per-step events"},
         "kernels_ms": {"quant_act_1x128": round(ms_act, 5), "quant_weight_128x128": round(ms_w, 5),
                        "gemm_blockscaled": round(ms_gemm, 5)},
         "gemm_tflops": round(gemm_tflops, 1),
@@ -274,9 +280,155 @@ def run_gpu(args, rank, world):
     if rank == 0 and not args.no_check:
         res["spot_check"] = spot_check(w, a_bits, b_bits, C)
 
+    if rank == 0 and not args.no_configs:
+        res["configs"] = config_throughput(fq, flush_l2)
+    if rank == 0 and not args.no_study:
+        res["accumulation_study"] = accumulation_study(fq)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w, a_bits, b_bits, budget_s=args.cpu_budget)
     return res
+
+
+# ------------------------------------------------------------------------------ other workloads
+
+def _time_ms(fn, reps, flush_l2):
+    """Mean device time of fn() over reps, L2 flushed before each (outside the events)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    tot = 0.0
+    for _ in range(reps):
+        flush_l2()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        e1.synchronize()
+        tot += e0.elapsed_time(e1)
+    return tot / reps
+
+
+def _dev_normal(shape, std, seed):
+    """Seeded normal bf16 samples generated on the device (timing-only inputs)."""
+    import torch
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    out = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+    flat = out.view(-1)
+    step = 1 << 26
+    for lo in range(0, flat.numel(), step):
+        hi = min(flat.numel(), lo + step)
+        flat[lo:hi] = (torch.randn(hi - lo, generator=g, device="cuda") * std).to(torch.bfloat16)
+    return out
+
+
+def config_throughput(fq, flush_l2, reps=10):
+    """Kernel times of the other workloads (inputs drawn on the device, same shapes and
+    distributions as the parity tests; their parity is covered by the GPU tests)."""
+    import torch
+    hbm, bf16_burst, _, _ = peaks()
+    fp8_peak = bf16_burst * FP8_PER_BF16
+    out = {}
+    # MoE prefill: 32 experts, Zipf routing, W [4096, 7168]
+    w = workloads.prefill()
+    off = torch.from_numpy(w.offsets).cuda()
+    A = _dev_normal((w.M, w.K), 1.0, 3001)
+    W = _dev_normal((w.experts, w.N, w.K), 0.006, 3002)
+    qA, sA = fq.quant_act_1x128(A, False)
+    qW, sW = fq.quant_weight_128x128(W, False)
+    C = torch.empty((w.M, w.N), dtype=torch.bfloat16, device="cuda")
+    t_a = _time_ms(lambda: fq.quant_act_1x128(A, False, out=(qA, sA)), reps, flush_l2)
+    t_w = _time_ms(lambda: fq.quant_weight_128x128(W, False, out=(qW, sW)), reps, flush_l2)
+    t_g = _time_ms(lambda: fq.gemm_grouped(qA, sA, qW, sW, off, out=C), reps, flush_l2)
+    tf = w.gemm_flops / (t_g * 1e-3) / 1e12
+    out["moe_prefill"] = {
+        "workload": w.name, "sum_M": w.M, "max_M": int(w.counts.max()), "min_M": int(w.counts.min()),
+        "gemm_ms": round(t_g, 4), "gemm_tflops": round(tf, 1), "gemm_frac_of_fp8_peak": round(tf / fp8_peak, 4),
+        "quant_act_gbs": round(w.M * w.K * (3 + 4 / 128) / (t_a * 1e-3) / 1e9, 1),
+        "quant_weight_gbs": round(W.numel() * (3 + 4 / 16384) / (t_w * 1e-3) / 1e9, 1)}
+    del A, W, qA, sA, qW, sW, C
+    # MoE decode: 64 experts, M_e ~ U{1..256}, W [7168, 2048] already FP8
+    w = workloads.decode()
+    off = torch.from_numpy(w.offsets).cuda()
+    A = _dev_normal((w.M, w.K), 1.0, 4001)
+    W = _dev_normal((w.experts, w.N, w.K), 0.006, 4002)
+    qA, sA = fq.quant_act_1x128(A, True)
+    qW, sW = fq.quant_weight_128x128(W, False)
+    C = torch.empty((w.M, w.N), dtype=torch.bfloat16, device="cuda")
+    t_g = _time_ms(lambda: fq.gemm_grouped(qA, sA, qW, sW, off, out=C), reps, flush_l2)
+    gemm_bytes = qW.numel() + sW.numel() * 4 + qA.numel() + sA.numel() * 4 + C.numel() * 2
+    out["moe_decode"] = {
+        "workload": w.name, "sum_M": w.M, "gemm_ms": round(t_g, 4),
+        "gemm_tflops": round(w.gemm_flops / (t_g * 1e-3) / 1e12, 1),
+        "gemm_gbs": round(gemm_bytes / (t_g * 1e-3) / 1e9, 1),
+        "gemm_frac_of_hbm": round(gemm_bytes / (t_g * 1e-3) / 1e9 / hbm, 4),
+        "algorithmic_bytes": int(gemm_bytes)}
+    del A, W, qA, sA, qW, sW, C
+    # wgrad: dY [7168, 16384] x X [2048, 16384], 1x128 both, fp32 out
+    w = workloads.wgrad()
+    A = _dev_normal((w.M, w.K), 1e-3, 5001)
+    B = _dev_normal((w.N, w.K), 1.0, 5002)
+    qA, sA = fq.quant_act_1x128(A, False)
+    qB, sB = fq.quant_act_1x128(B, False)
+    C = torch.empty((w.M, w.N), dtype=torch.float32, device="cuda")
+    t_a = _time_ms(lambda: fq.quant_act_1x128(A, False, out=(qA, sA)), reps, flush_l2)
+    t_g = _time_ms(lambda: fq.gemm_blockscaled(qA, sA, qB, sB, b_rowwise=True, out=C), reps, flush_l2)
+    tf = w.gemm_flops / (t_g * 1e-3) / 1e12
+    out["wgrad"] = {"workload": w.name, "gemm_ms": round(t_g, 4), "gemm_tflops": round(tf, 1),
+                    "gemm_frac_of_fp8_peak": round(tf / fp8_peak, 4),
+                    "quant_act_gbs": round(w.M * w.K * (3 + 4 / 128) / (t_a * 1e-3) / 1e9, 1)}
+    return out
+
+
+def accumulation_study(fq, rows_sampled=32):
+    """Error of the promoted GEMM and of the no-promotion GEMM versus K on the wgrad
+    workload (dY [7168, K] x X [2048, K], K = 4096 / 8192 / 16384 prefixes of one draw),
+    against the FP64 oracle on sampled rows.  Promoted: 1x128 codes (and, apples to
+    apples, the 1xK codes with their row scales repeated per group); no-promotion: 1xK
+    codes, one TMEM accumulator over all of K."""
+    import torch
+    import oracle
+    w = workloads.wgrad()
+    a_full, b_full = w.gen_a(), w.gen_b()
+    rows = np.sort(np.random.default_rng(5).choice(w.M, rows_sampled, replace=False))
+    rows_t = torch.from_numpy(rows).cuda()
+    res = []
+
+    def stats(Cs, C_ref, T):
+        d = np.abs(Cs.astype(np.float64) - C_ref)
+        r = d / np.maximum(T, 1e-300)
+        return {"max_rel_T": float(r.max()), "median_rel_T": float(np.median(r)),
+                "rel_frobenius": float(np.linalg.norm(d) / np.linalg.norm(C_ref))}
+
+    for K in (4096, 8192, 16384):
+        a_bits = np.ascontiguousarray(a_full[:, :K])
+        b_bits = np.ascontiguousarray(b_full[:, :K])
+        A, B = dev_bf16(a_bits), dev_bf16(b_bits)
+        G = K // 128
+        qa, sa = fq.quant_act_1x128(A, False)
+        qb, sb = fq.quant_act_1x128(B, False)
+        C_p = fq.gemm_blockscaled(qa, sa, qb, sb, out_dtype=torch.float32, b_rowwise=True)
+        qa1, sa1 = fq.quant_rowwise(A)
+        qb1, sb1 = fq.quant_rowwise(B)
+        C_n = fq.gemm_nopromo(qa1, sa1, qb1, sb1)
+        C_p1 = fq.gemm_blockscaled(qa1, sa1.expand(G, -1).contiguous(), qb1,
+                                   sb1.expand(G, -1).contiguous(), out_dtype=torch.float32,
+                                   b_rowwise=True)
+        torch.cuda.synchronize()
+        # oracle, from the bf16 inputs (never from the GPU's codes)
+        qa_r, sa_r = oracle.quant_act_1x128(a_bits[rows], False)
+        qb_r, sb_r = oracle.quant_act_1x128(b_bits, False)
+        C_ref, T = oracle.gemm_blockscaled_ref(qa_r, sa_r, qb_r, sb_r, b_rowwise=True)
+        qa1_r, sa1_r = oracle.quant_rowwise(a_bits[rows])
+        qb1_r, sb1_r = oracle.quant_rowwise(b_bits)
+        C1_ref, T1 = oracle.gemm_ref(oracle.dequant_rowwise(qa1_r, sa1_r),
+                                     oracle.dequant_rowwise(qb1_r, sb1_r))
+        res.append({"K": K,
+                    "promoted_1x128": stats(C_p[rows_t].cpu().numpy(), C_ref, T),
+                    "promoted_1xK_codes": stats(C_p1[rows_t].cpu().numpy(), C1_ref, T1),
+                    "no_promotion_1xK_codes": stats(C_n[rows_t].cpu().numpy(), C1_ref, T1)})
+        del A, B, qa, sa, qb, sb, C_p, qa1, sa1, qb1, sb1, C_n, C_p1
+    return {"rows_sampled": int(rows_sampled), "metric": "|C - C_ref| / sum_k|a b| (and Frobenius)",
+            "results": res}
 
 
 def kernel_rev() -> str:
@@ -373,6 +525,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-check", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' timings")
+    ap.add_argument("--no-study", action="store_true", help="skip the accumulation study")
     args = ap.parse_args()
 
     if args.impl == "reference":

@@ -23,12 +23,6 @@ using fp8q::GemmArgs;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-int device_sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
-  return n;
-}
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -60,21 +54,54 @@ int encode_operand(CUtensorMap* tm, const void* base, uint64_t K, uint64_t rows,
   return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
+// The promoted GEMMs launch one CTA per 128 x 256 tile.  The CTA-pair variant
+// (cta_group::2, 256 x 256 tiles, half of B per CTA) is correct but slower here: with
+// promotion every 128 K the TMEM accumulator has to be released once per group, and
+// the pair turns that release into a cross-CTA round trip (about 0.5 us against a
+// 0.26 us group), which the two TMEM buffers cannot hide.
+constexpr bool kPair = false;
+using Cfg = fp8q::GemmCfg<kPair>;
+
 template <bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16>
-int launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& args, int grid,
-                cudaStream_t stream) {
-  auto kern = fp8q::gemm_fp8_blockscaled_kernel<PROMOTE, ROW_B, GROUPED, OUT_BF16>;
-  static std::atomic<bool> configured[64];  // per instantiation, per device
-  const int smem = static_cast<int>(fp8q::SmemLayout::bytes);
+int launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& args,
+                int64_t work_units, cudaStream_t stream) {
+  auto kern = fp8q::gemm_fp8_blockscaled_kernel<kPair, PROMOTE, ROW_B, GROUPED, OUT_BF16>;
+  static std::atomic<int> max_units[64];  // per instantiation, per device: co-resident clusters
+  const int smem = static_cast<int>(Cfg::smem_bytes);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8Q_ERR_CUDA;
-  if (!configured[dev].load(std::memory_order_acquire)) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = Cfg::kCG;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(fp8q::kGemmThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int units = max_units[dev].load(std::memory_order_acquire);
+  if (units == 0) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return FP8Q_ERR_CUDA;
-    configured[dev].store(true, std::memory_order_release);
+    if (Cfg::kCG > 1 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess)
+      return FP8Q_ERR_CUDA;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return FP8Q_ERR_CUDA;
+    cfg.gridDim = dim3(static_cast<unsigned>(sms / Cfg::kCG * Cfg::kCG));
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0)
+      n = sms / Cfg::kCG;
+    units = n;
+    max_units[dev].store(units, std::memory_order_release);
   }
-  kern<<<grid, fp8q::kGemmThreads, smem, stream>>>(tmA, tmB, args);
+  const int64_t grid_units = work_units < units ? work_units : units;
+  if (grid_units <= 0) return FP8Q_OK;
+  cfg.gridDim = dim3(static_cast<unsigned>(grid_units * Cfg::kCG));
+  if (cudaLaunchKernelEx(&cfg, kern, tmA, tmB, args) != cudaSuccess) return FP8Q_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
@@ -95,13 +122,13 @@ int check_gemm_common(const uint8_t* A, const uint8_t* B, const void* C, int out
 
 template <bool PROMOTE, bool GROUPED>
 int dispatch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
-                         bool row_b, bool bf16, int grid, cudaStream_t st) {
+                  bool row_b, bool bf16, int64_t units, cudaStream_t st) {
   if (row_b) {
-    return bf16 ? launch_gemm<PROMOTE, true, GROUPED, true>(tmA, tmB, a, grid, st)
-                : launch_gemm<PROMOTE, true, GROUPED, false>(tmA, tmB, a, grid, st);
+    return bf16 ? launch_gemm<PROMOTE, true, GROUPED, true>(tmA, tmB, a, units, st)
+                : launch_gemm<PROMOTE, true, GROUPED, false>(tmA, tmB, a, units, st);
   }
-  return bf16 ? launch_gemm<PROMOTE, false, GROUPED, true>(tmA, tmB, a, grid, st)
-              : launch_gemm<PROMOTE, false, GROUPED, false>(tmA, tmB, a, grid, st);
+  return bf16 ? launch_gemm<PROMOTE, false, GROUPED, true>(tmA, tmB, a, units, st)
+              : launch_gemm<PROMOTE, false, GROUPED, false>(tmA, tmB, a, units, st);
 }
 
 }  // namespace
@@ -207,20 +234,16 @@ int fp8_gemm_blockscaled(const uint8_t* A, const float* sA, int64_t ld_sa, const
   if (ld_sa < M) return FP8Q_ERR_SHAPE;
   if (b_scale_mode == FP8Q_BSCALE_ROW1x128 && ld_sb < N) return FP8Q_ERR_SHAPE;
   if (!aligned(sA, 4) || !aligned(sB, 4)) return FP8Q_ERR_ALIGN;
-  const int sms = device_sm_count();
-  if (sms <= 0) return FP8Q_ERR_CUDA;
-
   CUtensorMap tmA, tmB;
-  if ((st = encode_operand(&tmA, A, K, M, lda, fp8q::kBM)) != FP8Q_OK) return st;
-  if ((st = encode_operand(&tmB, B, K, N, ldb, fp8q::kBN)) != FP8Q_OK) return st;
+  if ((st = encode_operand(&tmA, A, K, M, lda, 128)) != FP8Q_OK) return st;
+  if ((st = encode_operand(&tmB, B, K, N, ldb, Cfg::kBRows)) != FP8Q_OK) return st;
   GemmArgs a{};
   a.sA = sA; a.ld_sa = ld_sa; a.sB = sB; a.ld_sb = ld_sb; a.C = C; a.ldc = ldc;
   a.M = M; a.N = N; a.G = static_cast<int>(K / 128); a.m_offsets = nullptr; a.num_experts = 0;
-  const int64_t tiles = ((M + fp8q::kBM - 1) / fp8q::kBM) * ((N + fp8q::kBN - 1) / fp8q::kBN);
+  const int64_t tiles = ((M + Cfg::kTileM - 1) / Cfg::kTileM) * ((N + fp8q::kBN - 1) / fp8q::kBN);
   if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
   return dispatch_gemm<true, false>(tmA, tmB, a, b_scale_mode == FP8Q_BSCALE_ROW1x128,
-                                    out_dtype == FP8Q_OUT_BF16, grid, static_cast<cudaStream_t>(stream));
+                                    out_dtype == FP8Q_OUT_BF16, tiles, static_cast<cudaStream_t>(stream));
 }
 
 int fp8_gemm_grouped(const uint8_t* A, const float* sA, int64_t ld_sa, const uint8_t* W,
@@ -235,12 +258,9 @@ int fp8_gemm_grouped(const uint8_t* A, const float* sA, int64_t ld_sa, const uin
   if (ld_sa < max_sum_M) return FP8Q_ERR_SHAPE;
   if (!aligned(sA, 4) || !aligned(sW, 4) || !aligned(m_offsets, 4)) return FP8Q_ERR_ALIGN;
   if (static_cast<int64_t>(num_groups) * N > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  const int sms = device_sm_count();
-  if (sms <= 0) return FP8Q_ERR_CUDA;
-
   CUtensorMap tmA, tmB;
-  if ((st = encode_operand(&tmA, A, K, max_sum_M, K, fp8q::kBM)) != FP8Q_OK) return st;
-  if ((st = encode_operand(&tmB, W, K, static_cast<uint64_t>(num_groups) * N, K, fp8q::kBN)) != FP8Q_OK)
+  if ((st = encode_operand(&tmA, A, K, max_sum_M, K, 128)) != FP8Q_OK) return st;
+  if ((st = encode_operand(&tmB, W, K, static_cast<uint64_t>(num_groups) * N, K, Cfg::kBRows)) != FP8Q_OK)
     return st;
   GemmArgs a{};
   a.sA = sA; a.ld_sa = ld_sa; a.sB = sW; a.ld_sb = 0; a.C = C; a.ldc = N;
@@ -248,10 +268,9 @@ int fp8_gemm_grouped(const uint8_t* A, const float* sA, int64_t ld_sa, const uin
   a.m_offsets = m_offsets; a.num_experts = num_groups;
   // Upper bound on tiles (every group may add one partial m-tile) sizes the persistent grid.
   const int64_t nt = (N + fp8q::kBN - 1) / fp8q::kBN;
-  const int64_t bound = ((max_sum_M + fp8q::kBM - 1) / fp8q::kBM + num_groups) * nt;
+  const int64_t bound = ((max_sum_M + Cfg::kTileM - 1) / Cfg::kTileM + num_groups) * nt;
   if (bound > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  const int grid = static_cast<int>(bound < sms ? bound : sms);
-  return dispatch_gemm<true, true>(tmA, tmB, a, false, out_dtype == FP8Q_OUT_BF16, grid,
+  return dispatch_gemm<true, true>(tmA, tmB, a, false, out_dtype == FP8Q_OUT_BF16, bound,
                                    static_cast<cudaStream_t>(stream));
 }
 
@@ -263,18 +282,15 @@ int fp8_gemm_nopromo(const uint8_t* A, const float* sA, const uint8_t* B, const 
   if (st != FP8Q_OK) return st;
   if (!sA || !sB) return FP8Q_ERR_NULL;
   if (!aligned(sA, 4) || !aligned(sB, 4)) return FP8Q_ERR_ALIGN;
-  const int sms = device_sm_count();
-  if (sms <= 0) return FP8Q_ERR_CUDA;
   CUtensorMap tmA, tmB;
-  if ((st = encode_operand(&tmA, A, K, M, lda, fp8q::kBM)) != FP8Q_OK) return st;
-  if ((st = encode_operand(&tmB, B, K, N, ldb, fp8q::kBN)) != FP8Q_OK) return st;
+  if ((st = encode_operand(&tmA, A, K, M, lda, 128)) != FP8Q_OK) return st;
+  if ((st = encode_operand(&tmB, B, K, N, ldb, Cfg::kBRows)) != FP8Q_OK) return st;
   GemmArgs a{};
   a.sA = sA; a.ld_sa = 0; a.sB = sB; a.ld_sb = 0; a.C = C; a.ldc = ldc;
   a.M = M; a.N = N; a.G = static_cast<int>(K / 128); a.m_offsets = nullptr; a.num_experts = 0;
-  const int64_t tiles = ((M + fp8q::kBM - 1) / fp8q::kBM) * ((N + fp8q::kBN - 1) / fp8q::kBN);
+  const int64_t tiles = ((M + Cfg::kTileM - 1) / Cfg::kTileM) * ((N + fp8q::kBN - 1) / fp8q::kBN);
   if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-  return launch_gemm<false, false, false, false>(tmA, tmB, a, grid, static_cast<cudaStream_t>(stream));
+  return launch_gemm<false, false, false, false>(tmA, tmB, a, tiles, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -12,16 +12,27 @@
 // double-buffered TMEM accumulator: the tensor core fills buffer g+1 while the
 // epilogue warps drain buffer g.
 //
-// Roles (one 384-thread CTA per SM, persistent over output tiles):
-//   warp 0      TMA producer: A tile [128 x 128 B] and B tile [256 x 128 B] per
-//               K-group into a 4-stage shared-memory ring (128-byte swizzle).
-//   warp 1      TMEM owner + MMA issuer: 4 x tcgen05.mma kind::f8f6f4 (K = 32 each)
-//               per group into TMEM buffer (group parity), then tcgen05.commit to
-//               free the smem stage and to publish the partial.
+// Roles (384-thread CTAs, one per SM, persistent over output tiles):
+//   warp 0      TMA producer: per K-group, the CTA's A tile [128 rows x 128 B] and its
+//               B tile into a shared-memory ring (128-byte swizzle).
+//   warp 1      TMEM owner; in the MMA-issuing CTA also the MMA issuer: 4 x
+//               tcgen05.mma kind::f8f6f4 (K = 32 each) per group into TMEM buffer
+//               (group parity), then tcgen05.commit to free the smem stage and to
+//               publish the partial.
 //   warps 2-3   idle (they complete the first warpgroup).
 //   warps 4-11  promotion/epilogue: warp w reads TMEM lanes 32*(w%4).., columns
 //               128*((w-4)/4)..; per group: tcgen05.ld -> acc += P * scale in FP32
 //               registers; at tile end: convert and store C.
+//
+// PAIR = true: two CTAs of a cluster share a 256 x 256 output tile with
+// tcgen05 cta_group::2.  Each CTA loads its own 128 rows of A and 128 of the 256 rows
+// of B (32 KB per stage instead of 48 KB, so 6 stages fit), the even CTA issues the
+// M = 256 MMAs and its commits arrive on both CTAs' barriers; each CTA's TMEM holds
+// its 128 rows x 256 columns and its own epilogue promotes them; the odd CTA frees an
+// accumulator buffer with a remote arrive on the even CTA's barrier.  No TMA multicast:
+// every CTA loads its own operands.
+// PAIR = false (used by the promoted GEMMs): one CTA per 128 x 256 tile, B tile of 256
+// rows, 4 stages; every accumulator release is a local barrier arrive.
 //
 // Registers: the launch gives 168 per thread (3 warps per SM sub-partition).  The
 // first warpgroup gives registers back (setmaxnreg 56) and the two epilogue
@@ -39,14 +50,11 @@
 
 namespace fp8q {
 
-constexpr int kBM = 128, kBN = 256, kBK = 128;
-constexpr int kStages = 4;
+constexpr int kBN = 256, kBK = 128;
 constexpr int kEpiWarps = 8;
 constexpr int kEpiWarp0 = 4;                      // first epilogue warp (second warpgroup)
 constexpr int kGemmThreads = 32 * (kEpiWarp0 + kEpiWarps);
 constexpr int kRegsCtl = 56, kRegsEpi = 224;      // setmaxnreg split (see above)
-constexpr uint32_t kABytes = kBM * kBK;
-constexpr uint32_t kBBytes = kBN * kBK;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxGroups = 1024;
 
@@ -75,22 +83,33 @@ struct GemmArgs {
 
 constexpr uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-struct SmemLayout {
-  // byte offsets from the 1024-aligned base
-  static constexpr uint32_t a = 0;                                   // kStages x 16 KB
-  static constexpr uint32_t b = a + kStages * kABytes;               // kStages x 32 KB
+template <bool PAIR>
+struct GemmCfg {
+  static constexpr int kCG = PAIR ? 2 : 1;              // CTAs per MMA
+  static constexpr int kStages = PAIR ? 6 : 4;
+  static constexpr int kTileM = 128 * kCG;              // output rows per (pair) tile
+  static constexpr int kBRows = kBN / kCG;              // rows of B each CTA loads
+  static constexpr uint32_t kABytes = 128 * kBK;        // per CTA per stage
+  static constexpr uint32_t kBBytes = kBRows * kBK;
+  static constexpr uint32_t kStageTx = (kABytes + kBBytes) * kCG;  // bytes per full barrier phase
+  // accumulator release: every epilogue thread arrives (1 CTA); one remote arrive per
+  // epilogue warp of both CTAs (pair)
+  static constexpr uint32_t kTemptyArrivals = PAIR ? kCG * kEpiWarps : 32 * kEpiWarps;
+  // shared memory, byte offsets from the 1024-aligned base
+  static constexpr uint32_t a = 0;
+  static constexpr uint32_t b = a + kStages * kABytes;
   static constexpr uint32_t bars = b + kStages * kBBytes;
-  // barriers: full[S], empty[S], tfull[2], tempty[2], drain
-  static constexpr uint32_t n_bars = 2 * kStages + 5;
-  static constexpr uint32_t misc = align_up(bars + 8 * n_bars, 16);  // tmem slot, abort flag
-  static constexpr uint32_t sched = align_up(misc + 16, 16);         // int[kMaxGroups + 1]
+  static constexpr uint32_t n_bars = 2 * kStages + 5;   // full[S], empty[S], tfull[2], tempty[2], drain
+  static constexpr uint32_t misc = align_up(bars + 8 * n_bars, 16);   // tmem slot, abort flag
+  static constexpr uint32_t sched = align_up(misc + 16, 16);          // int[kMaxGroups + 1]
   static constexpr uint32_t sbrow = align_up(sched + 4 * (kMaxGroups + 1), 128);  // float[2][2][128]
   static constexpr uint32_t end = sbrow + 4 * 2 * 2 * 128;
-  static constexpr uint32_t bytes = end + 1024;                      // + base alignment slack
+  static constexpr uint32_t smem_bytes = end + 1024;                  // + base alignment slack
+  static_assert(a % 1024 == 0 && b % 1024 == 0 && kABytes % 1024 == 0 && kBBytes % 1024 == 0,
+                "swizzle atoms");
+  static_assert(sbrow % 16 == 0, "float4 reads of the scale slots");
+  static_assert(smem_bytes <= 232448, "fits the 227 KB opt-in shared memory");
 };
-static_assert(SmemLayout::a % 1024 == 0 && SmemLayout::b % 1024 == 0, "swizzle atoms");
-static_assert(SmemLayout::sbrow % 16 == 0, "float4 reads of the scale slots");
-static_assert(SmemLayout::bytes <= 232448, "fits the 227 KB opt-in shared memory");
 
 // Output tile of index t: first row of A, row bound for stores, first row of B (in the
 // stacked [E*N, K] weights), first output column, expert.
@@ -110,13 +129,13 @@ __device__ __forceinline__ void expert_rows(const GemmArgs& p, int e, int64_t& r
   r_end = en;
 }
 
-template <bool GROUPED>
+template <bool GROUPED, int TILE_M>
 __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& p, int mt_total, int nt_total,
                                             const int* sched) {
   Tile tl;
   if (!GROUPED) {
     const int mt = t % mt_total, nt = t / mt_total;
-    tl.row0 = static_cast<int64_t>(mt) * kBM;
+    tl.row0 = static_cast<int64_t>(mt) * TILE_M;
     tl.row_end = p.M;
     tl.col0 = static_cast<int64_t>(nt) * kBN;
     tl.brow0 = tl.col0;
@@ -131,10 +150,10 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& p, int mt_tot
     const int e = lo;
     int64_t r_begin, r_end;
     expert_rows(p, e, r_begin, r_end);
-    const int mte = static_cast<int>((r_end - r_begin + kBM - 1) / kBM);
+    const int mte = static_cast<int>((r_end - r_begin + TILE_M - 1) / TILE_M);
     const int local = t - sched[e];
     const int mt = local % mte, nt = local / mte;
-    tl.row0 = r_begin + static_cast<int64_t>(mt) * kBM;
+    tl.row0 = r_begin + static_cast<int64_t>(mt) * TILE_M;
     tl.row_end = r_end;
     tl.col0 = static_cast<int64_t>(nt) * kBN;
     tl.brow0 = static_cast<int64_t>(e) * p.N + tl.col0;
@@ -147,36 +166,42 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-template <bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16>
+template <bool PAIR, bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_fp8_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA,
                                 const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
+  using Cfg = GemmCfg<PAIR>;
+  constexpr int CG = Cfg::kCG;
+  constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar0 = sbase + SmemLayout::bars;
+  const uint32_t bar0 = sbase + Cfg::bars;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
-  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * kStages + b); };
-  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * kStages + 2 + b); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * kStages + 4);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SmemLayout::misc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SmemLayout::misc + 4);
-  int* sched = reinterpret_cast<int*>(smem + SmemLayout::sched);
-  float* sbrow = reinterpret_cast<float*>(smem + SmemLayout::sbrow);
+  auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * S + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * S + 2 + b); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * S + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::misc + 4);
+  int* sched = reinterpret_cast<int*>(smem + Cfg::sched);
+  float* sbrow = reinterpret_cast<float*>(smem + Cfg::sbrow);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.G;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;   // CTA 0 of a pair issues the MMAs
+  const bool mma_cta = rank == 0;
+  const int unit0 = blockIdx.x / CG, units = gridDim.x / CG;   // cluster index / count
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), 32 * kEpiWarps);
+      mbar_init(tempty_bar(b), Cfg::kTemptyArrivals);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -187,14 +212,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-    tmem_relinquish();
+    tmem_alloc<CG>(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish<CG>();
   }
 
   const int nt_total = static_cast<int>((p.N + kBN - 1) / kBN);
   int mt_total = 0, num_tiles = 0;
   if (!GROUPED) {
-    mt_total = static_cast<int>((p.M + kBM - 1) / kBM);
+    mt_total = static_cast<int>((p.M + Cfg::kTileM - 1) / Cfg::kTileM);
     num_tiles = mt_total * nt_total;
   } else {
     // per-expert tile counts, then an exclusive prefix (E is small)
@@ -202,7 +227,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int64_t rb, re;
       expert_rows(p, e, rb, re);
       const int64_t rows = re - rb;
-      sched[e + 1] = rows > 0 ? static_cast<int>((rows + kBM - 1) / kBM) * nt_total : 0;
+      sched[e + 1] = rows > 0 ? static_cast<int>((rows + Cfg::kTileM - 1) / Cfg::kTileM) * nt_total : 0;
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -212,101 +237,128 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if (PAIR) cluster_sync();       // the peer's barriers are initialised before any remote use
   tc_fence_after();
   if (GROUPED) num_tiles = sched[p.num_experts];
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp < kEpiWarp0) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      uint32_t it = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
-        const Tile tl = decode_tile<GROUPED>(t, p, mt_total, nt_total, sched);
-        for (int g = 0; g < G; ++g, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1u;
-          if (!mbar_wait(empty_bar(s), ph ^ 1u, kSiteProducer, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(full_bar(s), kABytes + kBBytes);
-          tma_load_2d(sbase + SmemLayout::a + s * kABytes, &tmA, full_bar(s), g * kBK,
-                      static_cast<int32_t>(tl.row0));
-          tma_load_2d(sbase + SmemLayout::b + s * kBBytes, &tmB, full_bar(s), g * kBK,
-                      static_cast<int32_t>(tl.brow0));
+    if (warp == 0) {
+      // ---------------------------------------------------------- TMA producer
+      if (lane == 0) {
+        uint32_t it = 0;
+        bool ok = true;
+        for (int t = unit0; ok && t < num_tiles; t += units) {
+          const Tile tl = decode_tile<GROUPED, Cfg::kTileM>(t, p, mt_total, nt_total, sched);
+          const int32_t arow = static_cast<int32_t>(tl.row0 + 128 * rank);
+          const int32_t brow = static_cast<int32_t>(tl.brow0 + Cfg::kBRows * rank);
+          for (int g = 0; g < G; ++g, ++it) {
+            const int s = it % S;
+            const uint32_t ph = (it / S) & 1u;
+            if (!mbar_wait(empty_bar(s), ph ^ 1u, kSiteProducer, abort_flag)) { ok = false; break; }
+            if (mma_cta) mbar_arrive_expect_tx(full_bar(s), Cfg::kStageTx);
+            const uint32_t dst_a = sbase + Cfg::a + s * Cfg::kABytes;
+            const uint32_t dst_b = sbase + Cfg::b + s * Cfg::kBBytes;
+            if (PAIR) {
+              const uint32_t fb = map_shared_rank(full_bar(s), 0);   // the MMA CTA's barrier
+              tma_load_2d_pair(dst_a, &tmA, fb, g * kBK, arow);
+              tma_load_2d_pair(dst_b, &tmB, fb, g * kBK, brow);
+            } else {
+              tma_load_2d(dst_a, &tmA, full_bar(s), g * kBK, arow);
+              tma_load_2d(dst_b, &tmB, full_bar(s), g * kBK, brow);
+            }
+          }
+        }
+        // Every issued load lands before the CTA can exit.  The MMA CTA watches its full
+        // barriers (bounded; loads finish on their own).  The other CTA's loads complete on
+        // the MMA CTA's barriers; in the normal path they were all consumed before the
+        // final cluster barrier, after an abort the teardown below waits a fixed while.
+        if (mma_cta) {
+          const uint32_t first = it > static_cast<uint32_t>(S) ? it - S : 0;
+          for (uint32_t j = first; j < it; ++j)
+            mbar_wait(full_bar(j % S), (j / S) & 1u, kSiteDrain, nullptr);
         }
       }
-      // Every issued load lands before the CTA can exit (bounded; loads finish on their own).
-      const uint32_t first = it > kStages ? it - kStages : 0;
-      for (uint32_t j = first; j < it; ++j)
-        mbar_wait(full_bar(j % kStages), (j / kStages) & 1u, kSiteDrain, nullptr);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(kBM, kBN);
-      uint32_t it = 0, acc_it = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
-        uint32_t buf = 0;
-        for (int g = 0; g < G; ++g, ++it) {
-          if (PROMOTE || g == 0) {
-            buf = acc_it & 1u;
-            if (!mbar_wait(tempty_bar(buf), ((acc_it >> 1) & 1u) ^ 1u, kSiteMmaEmpty, abort_flag)) {
+    } else if (warp == 1) {
+      // ---------------------------------------------------------- MMA issuer
+      if (lane == 0 && mma_cta) {
+        constexpr uint32_t idesc = idesc_e4m3_f32(Cfg::kTileM, kBN);
+        uint32_t it = 0, acc_it = 0;
+        bool ok = true;
+        for (int t = unit0; ok && t < num_tiles; t += units) {
+          uint32_t buf = 0;
+          for (int g = 0; g < G; ++g, ++it) {
+            if (PROMOTE || g == 0) {
+              buf = acc_it & 1u;
+              if (!mbar_wait(tempty_bar(buf), ((acc_it >> 1) & 1u) ^ 1u, kSiteMmaEmpty, abort_flag)) {
+                ok = false;
+                break;
+              }
+            }
+            const int s = it % S;
+            if (!mbar_wait(full_bar(s), (it / S) & 1u, kSiteMmaFull, abort_flag)) {
               ok = false;
               break;
             }
-          }
-          const int s = it % kStages;
-          if (!mbar_wait(full_bar(s), (it / kStages) & 1u, kSiteMmaFull, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t d = tmem_base + buf * kBN;
-          const uint32_t a_addr = sbase + SmemLayout::a + s * kABytes;
-          const uint32_t b_addr = sbase + SmemLayout::b + s * kBBytes;
+            tc_fence_after();
+            const uint32_t d = tmem_base + buf * kBN;
+            const uint32_t a_addr = sbase + Cfg::a + s * Cfg::kABytes;
+            const uint32_t b_addr = sbase + Cfg::b + s * Cfg::kBBytes;
 #pragma unroll
-          for (int kk = 0; kk < kBK / 32; ++kk) {
-            const uint32_t accumulate = PROMOTE ? (kk > 0) : (g > 0 || kk > 0);
-            mma_f8(d, smem_desc_k_sw128(a_addr + 32 * kk), smem_desc_k_sw128(b_addr + 32 * kk),
-                   idesc, accumulate);
-          }
-          mma_commit(empty_bar(s));
-          if (PROMOTE || g == G - 1) {
-            mma_commit(tfull_bar(buf));
-            ++acc_it;
+            for (int kk = 0; kk < kBK / 32; ++kk) {
+              const uint32_t accumulate = PROMOTE ? (kk > 0) : (g > 0 || kk > 0);
+              mma_f8<CG>(d, smem_desc_k_sw128(a_addr + 32 * kk), smem_desc_k_sw128(b_addr + 32 * kk),
+                         idesc, accumulate);
+            }
+            if (PAIR) mma_commit_pair(empty_bar(s), 0x3); else mma_commit<1>(empty_bar(s));
+            if (PROMOTE || g == G - 1) {
+              if (PAIR) mma_commit_pair(tfull_bar(buf), 0x3); else mma_commit<1>(tfull_bar(buf));
+              ++acc_it;
+            }
           }
         }
+        // All MMAs this thread issued complete before TMEM is released.
+        mma_commit<CG>(drain_bar);
+        mbar_wait(drain_bar, 0, kSiteDrain, nullptr);
       }
-      // All MMAs this thread issued complete before TMEM is released.
-      mma_commit(drain_bar);
-      mbar_wait(drain_bar, 0, kSiteDrain, nullptr);
     }
-  }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
     // ------------------------------------------------------------ promotion + epilogue
     const int ew = warp - kEpiWarp0;
     const int quad = warp & 3;              // TMEM lanes this warp may access
     const int set = ew >> 2;                // column half of the tile
-    const int row_in_tile = quad * 32 + lane;
+    const int row_in_tile = static_cast<int>(128 * rank) + quad * 32 + lane;
     const int tid_in_set = (ew & 3) * 32 + lane;
     float* sb_slots = sbrow + set * 2 * 128;
+    // Release of an accumulator buffer: each thread arrives on its own CTA's barrier; in
+    // a pair, one arrive per warp on the MMA CTA's barrier.
+    auto release = [&](uint32_t buf) {
+      tc_fence_before();
+      if (PAIR) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(map_shared_rank(tempty_bar(buf), 0));
+      } else {
+        mbar_arrive(tempty_bar(buf));
+      }
+    };
     // The epilogue never leaves its loops early: after an abort it keeps walking the
     // (uniform) tile/group structure without touching TMEM, so that every thread of a
     // column set reaches the same named barriers.
     uint32_t acc_it = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-      const Tile tl = decode_tile<GROUPED>(t, p, mt_total, nt_total, sched);
+    for (int t = unit0; t < num_tiles; t += units) {
+      const Tile tl = decode_tile<GROUPED, Cfg::kTileM>(t, p, mt_total, nt_total, sched);
       const int64_t m = tl.row0 + row_in_tile;
       const bool row_ok = m < tl.row_end;
       const int64_t n0 = tl.col0 + set * 128;
       const bool cols_ok = n0 < p.N;
-      float acc[128];
+      // acc[i] holds columns 2i, 2i+1 of this thread's row (packed FP32 pairs: the
+      // promotion runs on the f32x2 FMA path, two accumulations per instruction).
+      float2 acc[64];
 #pragma unroll
-      for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+      for (int j = 0; j < 64; ++j) acc[j] = make_float2(0.0f, 0.0f);
 
       if (PROMOTE) {
         const float* sB_tile = nullptr;
@@ -340,29 +392,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tc_fence_after();
             const uint32_t taddr =
                 tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + buf * kBN + set * 128;
-            const float sc = sa_cur * sb_cur;
+            const float2 sc2 = make_float2(sa_cur * sb_cur, sa_cur * sb_cur);
+            const float2 sa2 = make_float2(sa_cur, sa_cur);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint32_t r[32];
-              tmem_ld_32cols(taddr + c * 32, r);
+            for (int h = 0; h < 2; ++h) {
+              uint32_t r[64];
+              tmem_ld_64cols(taddr + h * 64, r);
               tmem_ld_wait();
-              if (c == 3) {
-                tc_fence_before();
-                mbar_arrive(tempty_bar(buf));
-              }
-              if (ROW_B) {
+              if (h == 1) release(buf);   // TMEM buffer free for group g+2
 #pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                  const float4 b4 = *reinterpret_cast<const float4*>(slot + c * 32 + j);
-                  acc[c * 32 + j + 0] = __fmaf_rn(__uint_as_float(r[j + 0]) * b4.x, sa_cur, acc[c * 32 + j + 0]);
-                  acc[c * 32 + j + 1] = __fmaf_rn(__uint_as_float(r[j + 1]) * b4.y, sa_cur, acc[c * 32 + j + 1]);
-                  acc[c * 32 + j + 2] = __fmaf_rn(__uint_as_float(r[j + 2]) * b4.z, sa_cur, acc[c * 32 + j + 2]);
-                  acc[c * 32 + j + 3] = __fmaf_rn(__uint_as_float(r[j + 3]) * b4.w, sa_cur, acc[c * 32 + j + 3]);
+              for (int j = 0; j < 64; j += 4) {
+                const float2 p0 = make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
+                const float2 p1 = make_float2(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+                float2& a0 = acc[(h * 64 + j) / 2];
+                float2& a1 = acc[(h * 64 + j) / 2 + 1];
+                if (ROW_B) {
+                  const float4 b4 = *reinterpret_cast<const float4*>(slot + h * 64 + j);
+                  a0 = __ffma2_rn(__fmul2_rn(p0, make_float2(b4.x, b4.y)), sa2, a0);
+                  a1 = __ffma2_rn(__fmul2_rn(p1, make_float2(b4.z, b4.w)), sa2, a1);
+                } else {
+                  a0 = __ffma2_rn(p0, sc2, a0);
+                  a1 = __ffma2_rn(p1, sc2, a1);
                 }
-              } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                  acc[c * 32 + j] = __fmaf_rn(__uint_as_float(r[j]), sc, acc[c * 32 + j]);
               }
             }
           }
@@ -383,18 +434,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_fence_after();
           const uint32_t taddr =
               tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + buf * kBN + set * 128;
+          const float2 sa2 = make_float2(sa, sa);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            tmem_ld_32cols(taddr + c * 32, r);
+          for (int h = 0; h < 2; ++h) {
+            uint32_t r[64];
+            tmem_ld_64cols(taddr + h * 64, r);
             tmem_ld_wait();
-            if (c == 3) {
-              tc_fence_before();
-              mbar_arrive(tempty_bar(buf));
-            }
+            if (h == 1) release(buf);
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              acc[c * 32 + j] = (__uint_as_float(r[j]) * sa) * slot[c * 32 + j];
+            for (int j = 0; j < 64; j += 2) {
+              const float2 pr = make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
+              const float2 sb2 = *reinterpret_cast<const float2*>(slot + h * 64 + j);
+              acc[(h * 64 + j) / 2] = __fmul2_rn(__fmul2_rn(pr, sa2), sb2);
+            }
           }
         }
         ++acc_it;
@@ -405,23 +457,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (OUT_BF16) {
           __nv_bfloat16* crow = reinterpret_cast<__nv_bfloat16*>(p.C) + m * p.ldc + n0;
 #pragma unroll
-          for (int j = 0; j < 128; j += 8) {
+          for (int j = 0; j < 64; j += 4) {
+            __nv_bfloat162 h0 = __float22bfloat162_rn(acc[j + 0]);
+            __nv_bfloat162 h1 = __float22bfloat162_rn(acc[j + 1]);
+            __nv_bfloat162 h2 = __float22bfloat162_rn(acc[j + 2]);
+            __nv_bfloat162 h3 = __float22bfloat162_rn(acc[j + 3]);
             uint4 o;
-            __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[j + 0], acc[j + 1]);
-            __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[j + 2], acc[j + 3]);
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[j + 4], acc[j + 5]);
-            __nv_bfloat162 h3 = __floats2bfloat162_rn(acc[j + 6], acc[j + 7]);
             o.x = *reinterpret_cast<uint32_t*>(&h0);
             o.y = *reinterpret_cast<uint32_t*>(&h1);
             o.z = *reinterpret_cast<uint32_t*>(&h2);
             o.w = *reinterpret_cast<uint32_t*>(&h3);
-            *reinterpret_cast<uint4*>(crow + j) = o;
+            *reinterpret_cast<uint4*>(crow + 2 * j) = o;
           }
         } else {
           float* crow = reinterpret_cast<float*>(p.C) + m * p.ldc + n0;
 #pragma unroll
-          for (int j = 0; j < 128; j += 4)
-            *reinterpret_cast<float4*>(crow + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+          for (int j = 0; j < 64; j += 2)
+            *reinterpret_cast<float4*>(crow + 2 * j) =
+                make_float4(acc[j].x, acc[j].y, acc[j + 1].x, acc[j + 1].y);
         }
       }
     }
@@ -430,10 +483,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
+  if (PAIR) {
+    // After an abort the other CTA's in-flight loads into this CTA's shared memory are
+    // not tracked by any local barrier: give them a fixed, generous time to land.
+    if (*abort_flag) {
+      const uint64_t t0 = globaltimer();
+      while (globaltimer() - t0 < 200000ull) {
+      }
+    }
+    __syncwarp();
+    cluster_sync();
+  }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc<CG>(tmem_base, kTmemCols);
+  }
+  if (PAIR) {
+    __syncwarp();
+    cluster_sync();               // neither CTA exits while its peer may still address it
   }
 }
 

@@ -31,9 +31,21 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
   return r;
 }
 
+// RN_f32(amax / 448) without a division instruction: 448 = 7 * 2^6, so 1/448 is not
+// exact, but with r = RN(1/448) one FMA residual correction gives the correctly rounded
+// quotient whenever the residual is representable (amax >= 2^-100; below that: divide).
+// The host check replays this for every positive bf16 amax.
+__device__ __forceinline__ float div448(float amax) {
+  if (amax < 0x1p-100f) return __fdiv_rn(amax, 448.0f);
+  const float r = 0x1.24924ap-9f;                 // RN(1/448)
+  const float q0 = __fmul_rn(amax, r);
+  const float e = __fmaf_rn(-q0, 448.0f, amax);
+  return __fmaf_rn(e, r, q0);
+}
+
 __device__ __forceinline__ float tile_scale(float amax, bool pow2) {
   if (amax == 0.0f) return 1.0f;
-  float s = __fdiv_rn(amax, 448.0f);
+  float s = div448(amax);
   if (pow2) {
     uint32_t b = __float_as_uint(s);
     const uint32_t mant = b & 0x7FFFFFu;
@@ -91,24 +103,51 @@ struct Quotient {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// max |x| over the 8 bf16 values of a 16-byte vector, returned as fp32.  On the
-// non-negative bf16 patterns (sign cleared) the unsigned integer order is the
-// value order, so the max is taken on the 16-bit patterns two at a time.
-__device__ __forceinline__ float amax8(const uint4& v) {
-  uint32_t m = __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
-  m = __vmaxu2(m, __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
-  const uint32_t hi = m >> 16, lo = m & 0xFFFFu;
-  return __uint_as_float((hi > lo ? hi : lo) << 16);
+// 8 bf16 -> 8 E4M3 bytes (uint2), each divided by the tile scale with quotient rule Q.
+template <typename Q>
+__device__ __forceinline__ uint2 quant8_with(const uint4& v, Q q) {
+  uint2 o;
+  o.x = cvt_e4m3x2(q(bf16lo(v.x)), q(bf16hi(v.x))) | (cvt_e4m3x2(q(bf16lo(v.y)), q(bf16hi(v.y))) << 16);
+  o.y = cvt_e4m3x2(q(bf16lo(v.z)), q(bf16hi(v.z))) | (cvt_e4m3x2(q(bf16lo(v.w)), q(bf16hi(v.w))) << 16);
+  return o;
 }
 
-// 8 bf16 -> 8 E4M3 bytes (uint2), all divided by the tile scale.
-__device__ __forceinline__ uint2 quant8(const uint4& v, const Quotient& qd) {
-  uint2 o;
-  o.x = cvt_e4m3x2(qd(bf16lo(v.x)), qd(bf16hi(v.x))) |
-        (cvt_e4m3x2(qd(bf16lo(v.y)), qd(bf16hi(v.y))) << 16);
-  o.y = cvt_e4m3x2(qd(bf16lo(v.z)), qd(bf16hi(v.z))) |
-        (cvt_e4m3x2(qd(bf16lo(v.w)), qd(bf16hi(v.w))) << 16);
-  return o;
+// Quantize NV vectors of 8 bf16 with one tile scale; the quotient rule is chosen once.
+template <int NV>
+__device__ __forceinline__ void quant_vectors(const uint4 (&v)[NV], const Quotient& qd, uint2 (&o)[NV]) {
+  if (qd.mode == kExactRcp) {
+    const float r = qd.r;
+    auto f = [r](float x) { return __fmul_rn(x, r); };
+#pragma unroll
+    for (int j = 0; j < NV; ++j) o[j] = quant8_with(v[j], f);
+  } else if (qd.mode == kCorrected) {
+    const float r = qd.r, sc = qd.s;
+    auto f = [r, sc](float x) {
+      const float q0 = __fmul_rn(x, r);
+      const float e = __fmaf_rn(-q0, sc, x);
+      return copysignf(__fmaf_rn(e, r, q0), x);
+    };
+#pragma unroll
+    for (int j = 0; j < NV; ++j) o[j] = quant8_with(v[j], f);
+  } else {
+    const float sc = qd.s;
+    auto f = [sc](float x) { return __fdiv_rn(x, sc); };
+#pragma unroll
+    for (int j = 0; j < NV; ++j) o[j] = quant8_with(v[j], f);
+  }
+}
+
+// max |x| over NV vectors of 8 bf16 (fold the 16-bit patterns first, convert once).
+template <int NV>
+__device__ __forceinline__ float amax_vectors(const uint4 (&v)[NV]) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    m = __vmaxu2(m, __vmaxu2(v[j].x & 0x7FFF7FFFu, v[j].y & 0x7FFF7FFFu));
+    m = __vmaxu2(m, __vmaxu2(v[j].z & 0x7FFF7FFFu, v[j].w & 0x7FFF7FFFu));
+  }
+  const uint32_t hi = m >> 16, lo = m & 0xFFFFu;
+  return __uint_as_float((hi > lo ? hi : lo) << 16);
 }
 
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
@@ -125,47 +164,41 @@ __device__ __forceinline__ void stg_u2(void* p, uint2 v) {
 
 // ---------------------------------------------------------------- 1x128 activation tiles
 //
-// Grid (ceil(M / 64), G).  A block of 8 warps covers 64 rows of one 128-column group:
-// each half-warp owns one row's group (16 lanes x 8 bf16 = 256 contiguous bytes), each
-// warp walks 4 pairs of rows with all four loads issued before any math.  The amax is a
-// 4-step xor-shuffle inside the half-warp; lane 0 of the half writes the scale, so the
-// scales of consecutive rows of a group land in consecutive words.
-constexpr int kActRowsPerWarp = 8;
-constexpr int kActWarps = 8;
-constexpr int kActRowsPerBlock = kActRowsPerWarp * kActWarps;
+// Grid (ceil(M / 64), G), 256 threads.  A team of 4 lanes owns one row's 128-element
+// group: lane l of the team holds the 16-byte chunks l, l+4, l+8, l+12 (so each load
+// instruction reads 64 contiguous bytes per team), all four loads in flight before any
+// arithmetic.  The amax needs two xor-shuffles inside the team; the scale and its
+// reciprocal are computed once per lane for 32 elements.  A warp covers 8 consecutive
+// rows of one group, so lane 0 of each team writes 8 consecutive scale words.
+constexpr int kActRowsPerBlock = 64;
 
 template <bool POW2>
 __global__ void __launch_bounds__(256) quant_act_1x128_kernel(const uint16_t* __restrict__ x,
                                                               int64_t M, int64_t ldx,
                                                               uint8_t* __restrict__ q, int64_t ldq,
                                                               float* __restrict__ s, int64_t lds) {
-  const int lane = threadIdx.x & 31;
-  const int half = lane >> 4, sub = lane & 15;
-  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int l4 = lane & 3;
   const int64_t g = blockIdx.y;
-  const int64_t m_first = static_cast<int64_t>(blockIdx.x) * kActRowsPerBlock + warp * kActRowsPerWarp + half;
-  constexpr int U = kActRowsPerWarp / 2;
+  const int64_t m = static_cast<int64_t>(blockIdx.x) * kActRowsPerBlock + warp * 8 + (lane >> 2);
+  const bool valid = m < M;
+  const uint16_t* src = x + m * ldx + g * 128 + l4 * 8;
 
-  uint4 v[U];
+  uint4 v[4];
 #pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const int64_t m = m_first + 2 * u;
-    v[u] = (m < M) ? ldg_stream(x + m * ldx + g * 128 + sub * 8) : make_uint4(0, 0, 0, 0);
-  }
+  for (int j = 0; j < 4; ++j) v[j] = valid ? ldg_stream(src + 32 * j) : make_uint4(0, 0, 0, 0);
+  float a = amax_vectors(v);
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+  const float sc = tile_scale(a, POW2);
+  if (valid) {
+    const Quotient qd(sc);
+    uint2 o[4];
+    quant_vectors(v, qd, o);
+    uint8_t* dst = q + m * ldq + g * 128 + l4 * 8;
 #pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const int64_t m = m_first + 2 * u;
-    float a = amax8(v[u]);
-    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 8));
-    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
-    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
-    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
-    const float sc = tile_scale(a, POW2);
-    if (m < M) {
-      const Quotient qd(sc);
-      stg_u2(q + m * ldq + g * 128 + sub * 8, quant8(v[u], qd));
-      if (sub == 0) s[g * lds + m] = sc;
-    }
+    for (int j = 0; j < 4; ++j) stg_u2(dst + 32 * j, o[j]);
+    if (l4 == 0) s[g * lds + m] = sc;
   }
 }
 
@@ -190,9 +223,7 @@ __global__ void __launch_bounds__(256) quant_weight_128x128_kernel(const uint16_
   uint4 v[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) v[j] = ldg_stream(base + static_cast<int64_t>(16 * j) * ldw);
-  float a = 0.0f;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) a = fmaxf(a, amax8(v[j]));
+  float a = amax_vectors(v);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
   if ((t & 31) == 0) red[t >> 5] = a;
@@ -203,8 +234,10 @@ __global__ void __launch_bounds__(256) quant_weight_128x128_kernel(const uint16_
   const float sc = tile_scale(a, POW2);
   const Quotient qd(sc);
   uint8_t* qb = q + (nb * 128 + r0) * ldq + g * 128 + c * 8;
+  uint2 o[8];
+  quant_vectors(v, qd, o);
 #pragma unroll
-  for (int j = 0; j < 8; ++j) stg_u2(qb + static_cast<int64_t>(16 * j) * ldq, quant8(v[j], qd));
+  for (int j = 0; j < 8; ++j) stg_u2(qb + static_cast<int64_t>(16 * j) * ldq, o[j]);
   if (t == 0) s[nb * G + g] = sc;
 }
 
@@ -223,7 +256,10 @@ __global__ void __launch_bounds__(256) quant_rowwise_kernel(const uint16_t* __re
   const uint16_t* xr = x + m * ldx;
   float a = 0.0f;
   for (int64_t k = static_cast<int64_t>(threadIdx.x) * 8; k < K; k += 256 * 8)
-    a = fmaxf(a, amax8(ldg_stream(xr + k)));
+  {
+    const uint4 v[1] = {ldg_stream(xr + k)};
+    a = fmaxf(a, amax_vectors(v));
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
@@ -233,8 +269,12 @@ __global__ void __launch_bounds__(256) quant_rowwise_kernel(const uint16_t* __re
   for (int i = 1; i < 8; ++i) a = fmaxf(a, red[i]);
   const float sc = tile_scale(a, POW2);
   const Quotient qd(sc);
-  for (int64_t k = static_cast<int64_t>(threadIdx.x) * 8; k < K; k += 256 * 8)
-    stg_u2(q + m * ldq + k, quant8(ldg_stream(xr + k), qd));
+  for (int64_t k = static_cast<int64_t>(threadIdx.x) * 8; k < K; k += 256 * 8) {
+    const uint4 v[1] = {ldg_stream(xr + k)};
+    uint2 o[1];
+    quant_vectors(v, qd, o);
+    stg_u2(q + m * ldq + k, o[0]);
+  }
   if (threadIdx.x == 0) s[m] = sc;
 }
 

@@ -12,7 +12,8 @@
  *   - otherwise a quotient of the same sign with magnitude <= 2^-10 (E4M3 rounds
  *     both to a signed zero).
  * It also checks the kernels' power-of-two rounding of s (an exponent bit trick)
- * against the definition "smallest power of two >= s".
+ * against the definition "smallest power of two >= s", and their amax / 448 (a
+ * corrected reciprocal) against IEEE division for every positive bf16 amax.
  * Exit status 0 and "ok" on success.
  */
 #include <math.h>
@@ -42,8 +43,22 @@ static float def_pow2(float s) {
     return (float)(f == 0.5 ? (double)s : ldexp(1.0, ex));
 }
 
+/* the kernels' amax / 448: RN(1/448) and one FMA residual correction (tiny amax divide) */
+static float kernel_div448(float amax) {
+    if (amax < 0x1p-100f) return amax / 448.0f;
+    const float r = 0x1.24924ap-9f;
+    float q0 = amax * r;
+    float e = fmaf(-q0, 448.0f, amax);
+    return fmaf(e, r, q0);
+}
+
 int main(void) {
-    long long bad = 0, checked = 0, bad_pow2 = 0;
+    long long bad = 0, checked = 0, bad_pow2 = 0, bad_div448 = 0;
+    if (0x1.24924ap-9f != 1.0f / 448.0f) { printf("RN(1/448) constant is wrong\n"); return 1; }
+    for (int ab = 1; ab < 0x7F80; ++ab) {      /* every positive finite bf16 amax */
+        float amax = f_of((uint32_t)ab << 16);
+        if (b_of(kernel_div448(amax)) != b_of(amax / 448.0f)) ++bad_div448;
+    }
 #pragma omp parallel for schedule(dynamic, 64) reduction(+ : bad, checked, bad_pow2)
     for (int ab = 1; ab < 0x7F80; ++ab) {
         float amax = f_of((uint32_t)ab << 16);
@@ -83,7 +98,8 @@ int main(void) {
             }
         }
     }
-    printf("checked %lld quotients: %lld mismatches, %lld pow2 mismatches\n", checked, bad, bad_pow2);
-    if (bad == 0 && bad_pow2 == 0) { printf("ok\n"); return 0; }
+    printf("checked %lld quotients: %lld mismatches, %lld pow2 mismatches, %lld amax/448 mismatches\n",
+           checked, bad, bad_pow2, bad_div448);
+    if (bad == 0 && bad_pow2 == 0 && bad_div448 == 0) { printf("ok\n"); return 0; }
     return 1;
 }
