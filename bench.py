@@ -431,6 +431,34 @@ def accumulation_study(fq, rows_sampled=32):
             "results": res}
 
 
+def profile_case(name: str, launches: int = 3):
+    """A few launches of one workload's kernels on device-drawn inputs (for ncu captures)."""
+    import torch
+    import fp8_fine_grained_weight_b200 as fq
+    w = workloads.ALL[name]()
+    if w.experts:
+        off = torch.from_numpy(w.offsets).cuda()
+        A = _dev_normal((w.M, w.K), w.a_std, 7001)
+        W = _dev_normal((w.experts, w.N, w.K), w.b_std, 7002)
+        qA, sA = fq.quant_act_1x128(A, w.pow2_a)
+        qW, sW = fq.quant_weight_128x128(W, w.pow2_b)
+        C = torch.empty((w.M, w.N), dtype=torch.bfloat16, device="cuda")
+        run = lambda: fq.gemm_grouped(qA, sA, qW, sW, off, out=C)
+    else:
+        A = _dev_normal((w.M, w.K), w.a_std, 7001)
+        B = _dev_normal((w.N, w.K), w.b_std, 7002)
+        qA, sA = fq.quant_act_1x128(A, w.pow2_a)
+        qB, sB = fq.quant_act_1x128(B, w.pow2_b) if w.b_rowwise else fq.quant_weight_128x128(B, w.pow2_b)
+        C = torch.empty((w.M, w.N), dtype=torch.float32 if w.out_fp32 else torch.bfloat16, device="cuda")
+        run = lambda: fq.gemm_blockscaled(qA, sA, qB, sB, b_rowwise=w.b_rowwise, out=C)
+    for _ in range(launches):
+        run()
+    torch.cuda.synchronize()
+    if fq.device_error():
+        raise RuntimeError("device error word set")
+    print(json.dumps({"profile_case": w.name, "launches": launches}), flush=True)
+
+
 def kernel_rev() -> str:
     """Short hash of the kernel sources, to tie stored ncu counters to the code they measured."""
     import hashlib
@@ -520,14 +548,23 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="dense", choices=["tiny", "dense", "wgrad"])
+    ap.add_argument("--workload", default="dense", choices=["tiny", "dense", "wgrad"],
+                    help="the dense workload timed as one step (the bench line)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-check", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' timings")
     ap.add_argument("--no-study", action="store_true", help="skip the accumulation study")
+    ap.add_argument("--profile-case", choices=["tiny", "dense", "prefill", "decode", "wgrad"],
+                    help="only run a few GEMM launches of one workload (for ncu) and exit")
     args = ap.parse_args()
+
+    if args.profile_case:
+        import torch
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        profile_case(args.profile_case)
+        return
 
     if args.impl == "reference":
         if int(os.environ.get("RANK", "0")) != 0:
