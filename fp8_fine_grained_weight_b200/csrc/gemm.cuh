@@ -19,7 +19,10 @@
 //               tcgen05.mma kind::f8f6f4 (K = 32 each) per group into TMEM buffer
 //               (group parity), then tcgen05.commit to free the smem stage and to
 //               publish the partial.
-//   warps 2-3   idle (they complete the first warpgroup).
+//   warp 2      scale producer: for every group, ahead of the epilogue, copies the
+//               tile's 128 row scales of A and its B scales (2 block scales, or 256
+//               column scales) into an 8-slot shared-memory ring with cp.async.
+//   warp 3      idle (it completes the first warpgroup).
 //   warps 4-11  promotion/epilogue: warp w reads TMEM lanes 32*(w%4).., columns
 //               128*((w-4)/4)..; per group: tcgen05.ld -> acc += P * scale in FP32
 //               registers; at tile end: convert and store C.
@@ -64,7 +67,8 @@ enum : unsigned int {
   kSiteMmaFull = 2,
   kSiteMmaEmpty = 3,
   kSiteEpilogue = 4,
-  kSiteDrain = 5
+  kSiteDrain = 5,
+  kSiteScales = 6
 };
 
 struct GemmArgs {
@@ -99,15 +103,19 @@ struct GemmCfg {
   static constexpr uint32_t a = 0;
   static constexpr uint32_t b = a + kStages * kABytes;
   static constexpr uint32_t bars = b + kStages * kBBytes;
-  static constexpr uint32_t n_bars = 2 * kStages + 5;   // full[S], empty[S], tfull[2], tempty[2], drain
+  static constexpr int kScaleSlots = 8;                  // scale ring depth (groups)
+  static constexpr uint32_t kSlotFloats = 128 + 256;     // A row scales + B scales
+  // full[S], empty[S], tfull[2], tempty[2], drain, sfull[R], sempty[R]
+  static constexpr uint32_t n_bars = 2 * kStages + 5 + 2 * kScaleSlots;
   static constexpr uint32_t misc = align_up(bars + 8 * n_bars, 16);   // tmem slot, abort flag
   static constexpr uint32_t sched = align_up(misc + 16, 16);          // int[kMaxGroups + 1]
   static constexpr uint32_t sbrow = align_up(sched + 4 * (kMaxGroups + 1), 128);  // float[2][2][128]
-  static constexpr uint32_t end = sbrow + 4 * 2 * 2 * 128;
+  static constexpr uint32_t sring = align_up(sbrow + 4 * 2 * 2 * 128, 128);  // float[R][kSlotFloats]
+  static constexpr uint32_t end = sring + 4 * kScaleSlots * kSlotFloats;
   static constexpr uint32_t smem_bytes = end + 1024;                  // + base alignment slack
   static_assert(a % 1024 == 0 && b % 1024 == 0 && kABytes % 1024 == 0 && kBBytes % 1024 == 0,
                 "swizzle atoms");
-  static_assert(sbrow % 16 == 0, "float4 reads of the scale slots");
+  static_assert(sbrow % 16 == 0 && sring % 16 == 0, "float4 reads of the scale slots");
   static_assert(smem_bytes <= 232448, "fits the 227 KB opt-in shared memory");
 };
 
@@ -183,6 +191,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * S + b); };
   auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * S + 2 + b); };
   const uint32_t drain_bar = bar0 + 8u * (2 * S + 4);
+  constexpr int R = Cfg::kScaleSlots;
+  auto sfull_bar = [&](int r) { return bar0 + 8u * (2 * S + 5 + r); };
+  auto sempty_bar = [&](int r) { return bar0 + 8u * (2 * S + 5 + R + r); };
+  float* sring = reinterpret_cast<float*>(smem + Cfg::sring);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::misc + 4);
   int* sched = reinterpret_cast<int*>(smem + Cfg::sched);
@@ -204,6 +216,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(tempty_bar(b), Cfg::kTemptyArrivals);
     }
     mbar_init(drain_bar, 1);
+    for (int r = 0; r < R; ++r) {
+      mbar_init(sfull_bar(r), 32);                 // one cp.async arrival per producer lane
+      mbar_init(sempty_bar(r), 32 * kEpiWarps);    // every epilogue thread frees the slot
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -322,6 +338,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mma_commit<CG>(drain_bar);
         mbar_wait(drain_bar, 0, kSiteDrain, nullptr);
       }
+    } else if (warp == 2 && PROMOTE) {
+      // ---------------------------------------------------------- scale producer
+      // Slot layout: [0, 128) A scales of this CTA's 128 rows; [128, 384) B scales: the
+      // 256 column scales (ROW mode) or, for 128x128 weight blocks, the two blocks'.
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = unit0; ok && t < num_tiles; t += units) {
+        const Tile tl = decode_tile<GROUPED, Cfg::kTileM>(t, p, mt_total, nt_total, sched);
+        const int64_t r0 = tl.row0 + 128 * rank;
+        const float* sB_tile =
+            ROW_B ? nullptr : p.sB + (static_cast<int64_t>(tl.expert) * (p.N / 128) + tl.col0 / 128) * G;
+        for (int g = 0; g < G; ++g, ++it) {
+          const int r = it % R;
+          if (!mbar_wait(sempty_bar(r), ((it / R) & 1u) ^ 1u, kSiteScales, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t slot = sbase + Cfg::sring + 4u * Cfg::kSlotFloats * r;
+          const float* sa_g = p.sA + static_cast<int64_t>(g) * p.ld_sa;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int64_t m = r0 + 32 * j + lane;
+            cp_async_4(slot + 4u * (32 * j + lane), sa_g + (m < tl.row_end ? m : 0), m < tl.row_end);
+          }
+          if (ROW_B) {
+            const float* sb_g = p.sB + static_cast<int64_t>(g) * p.ld_sb;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int64_t n = tl.col0 + 32 * j + lane;
+              cp_async_4(slot + 4u * (128 + 32 * j + lane), sb_g + (n < p.N ? n : 0), n < p.N);
+            }
+          } else if (lane < 2) {
+            const bool v = tl.col0 + 128 * lane < p.N;
+            cp_async_4(slot + 4u * (128 + lane), sB_tile + (v ? lane * G + g : 0), v);
+          }
+          cp_async_arrive(sfull_bar(r));
+        }
+      }
+      cp_async_wait_all();     // no copy into shared memory outlives the CTA
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
@@ -361,31 +416,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int j = 0; j < 64; ++j) acc[j] = make_float2(0.0f, 0.0f);
 
       if (PROMOTE) {
-        const float* sB_tile = nullptr;
-        if (!ROW_B)
-          sB_tile = p.sB + (static_cast<int64_t>(tl.expert) * (p.N / 128) + n0 / 128) * G;
-        auto load_sa = [&](int g) -> float {
-          return row_ok ? __ldg(p.sA + static_cast<int64_t>(g) * p.ld_sa + m) : 0.0f;
-        };
-        auto load_sb = [&](int g) -> float {
-          if (ROW_B) {
-            const int64_t n = n0 + tid_in_set;
-            return cols_ok ? __ldg(p.sB + static_cast<int64_t>(g) * p.ld_sb + n) : 0.0f;
-          }
-          return cols_ok ? __ldg(sB_tile + g) : 0.0f;
-        };
-        float sa_cur = load_sa(0), sb_cur = load_sb(0);
         for (int g = 0; g < G; ++g) {
-          const bool more = g + 1 < G;
-          const float sa_nxt = more ? load_sa(g + 1) : 0.0f;
-          const float sb_nxt = more ? load_sb(g + 1) : 0.0f;
-          // ROW mode: the set's 128 column scales of this group go through a 2-slot
-          // ring that alternates with every group of every tile.
-          float* slot = sb_slots + (acc_it & 1u) * 128;
-          if (ROW_B) {
-            slot[tid_in_set] = sb_cur;
-            named_bar_sync(1 + set, 128);
-          }
+          // This group's scales, staged by the scale producer (the ring advances with
+          // every group of every tile, in the same order as acc_it).
+          const int r = acc_it % R;
+          const float* slot = sring + Cfg::kSlotFloats * r;
+          if (ok) ok = mbar_wait(sfull_bar(r), (acc_it / R) & 1u, kSiteScales, abort_flag);
+          const float sa_cur = slot[quad * 32 + lane];
+          const float sb_cur = ROW_B ? 0.0f : slot[128 + set];
+          const float* sbv = slot + 128 + set * 128;        // ROW mode column scales
           const uint32_t buf = acc_it & 1u;
           if (ok) ok = mbar_wait(tfull_bar(buf), (acc_it >> 1) & 1u, kSiteEpilogue, abort_flag);
           if (ok) {
@@ -407,7 +446,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 float2& a0 = acc[(h * 64 + j) / 2];
                 float2& a1 = acc[(h * 64 + j) / 2 + 1];
                 if (ROW_B) {
-                  const float4 b4 = *reinterpret_cast<const float4*>(slot + h * 64 + j);
+                  const float4 b4 = *reinterpret_cast<const float4*>(sbv + h * 64 + j);
                   a0 = __ffma2_rn(__fmul2_rn(p0, make_float2(b4.x, b4.y)), sa2, a0);
                   a1 = __ffma2_rn(__fmul2_rn(p1, make_float2(b4.z, b4.w)), sa2, a1);
                 } else {
@@ -417,9 +456,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               }
             }
           }
+          mbar_arrive(sempty_bar(r));   // scales of this group consumed
           ++acc_it;
-          sa_cur = sa_nxt;
-          sb_cur = sb_nxt;
         }
       } else {
         // no promotion: one accumulator over all of K, scaled once by sA[m] * sB[n]
