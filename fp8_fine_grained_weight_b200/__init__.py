@@ -36,6 +36,9 @@ SIGNATURES = {
     "fp8q_quant_rowwise": (_i32, [_vp, _i64, _i64, _i64, _vp, _i64, _vp, _i32, _vp]),
     "fp8_gemm_blockscaled": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _i32, _vp, _i32,
                                     _i64, _i64, _i64, _i64, _i64, _i64, _vp]),
+    "fp8_gemm_blockscaled_ws": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _i32, _vp, _i32,
+                                       _i64, _i64, _i64, _i64, _i64, _i64, _vp, ctypes.c_size_t, _vp]),
+    "fp8_gemm_workspace_size": (_i32, [_i64, _i64, _i64, ctypes.POINTER(ctypes.c_size_t)]),
     "fp8_gemm_grouped": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _i32, _vp, _i32,
                                 _i64, _i64, _i64, _vp]),
     "fp8_gemm_nopromo": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _vp]),
@@ -158,13 +161,37 @@ def _out_code(out_dtype) -> int:
     raise TypeError("out_dtype must be torch.bfloat16 or torch.float32")
 
 
+_WORKSPACE = {}
+
+
+def workspace_bytes(M: int, N: int, K: int) -> int:
+    """Device workspace the dense GEMM can use to split its last wave (0 if none)."""
+    n = ctypes.c_size_t(0)
+    _call("fp8_gemm_workspace_size", M, N, K, ctypes.byref(n))
+    return int(n.value)
+
+
+def _workspace(device, nbytes: int) -> torch.Tensor:
+    """A per-device scratch buffer of at least nbytes, grown on demand (never shrunk).
+    Calls on one stream reuse it; concurrent streams should pass their own."""
+    key = torch.device(device).index
+    ws = _WORKSPACE.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        _WORKSPACE[key] = ws
+    return ws
+
+
 def gemm_blockscaled(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor,
                      out_dtype=torch.bfloat16, b_rowwise: bool = False,
-                     out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                     out: Optional[torch.Tensor] = None, split_k: bool = True,
+                     workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
     """C = A B^T with per-128-K promotion.
 
     qa uint8 [M, K]; sa fp32 [K/128, >= M]; qb uint8 [N, K];
     sb fp32 [N/128, K/128] (128x128 blocks) or, with ``b_rowwise``, [K/128, >= N].
+    ``split_k``: split the last partial wave of tiles along K (uses a device workspace:
+    ``workspace`` if given, else a cached per-device buffer).
     """
     qa, qb = _u8(qa), _u8(qb)
     _need(qa, torch.uint8, "qa", 2)
@@ -177,10 +204,17 @@ def gemm_blockscaled(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: t
         raise ValueError("qa and qb disagree on K")
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=qa.device)
-    _call("fp8_gemm_blockscaled", qa.data_ptr(), sa.data_ptr(), sa.stride(0), qb.data_ptr(),
+    ws_ptr, ws_len = None, 0
+    if split_k and M > 0:
+        need = workspace_bytes(M, N, K)
+        if need:
+            ws = workspace if workspace is not None else _workspace(qa.device, need)
+            if ws.numel() * ws.element_size() >= need:
+                ws_ptr, ws_len = ws.data_ptr(), ws.numel() * ws.element_size()
+    _call("fp8_gemm_blockscaled_ws", qa.data_ptr(), sa.data_ptr(), sa.stride(0), qb.data_ptr(),
           sb.data_ptr(), sb.stride(0) if b_rowwise else 0,
           BSCALE_ROW if b_rowwise else BSCALE_BLOCK, out.data_ptr(), _out_code(out.dtype),
-          M, N, K, qa.stride(0), qb.stride(0), out.stride(0), _stream(qa))
+          M, N, K, qa.stride(0), qb.stride(0), out.stride(0), ws_ptr, ws_len, _stream(qa))
     return out
 
 

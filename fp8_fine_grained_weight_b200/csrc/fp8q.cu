@@ -63,46 +63,81 @@ constexpr bool kPair = false;
 using Cfg = fp8q::GemmCfg<kPair>;
 
 template <bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16>
-int launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& args,
-                int64_t work_units, cudaStream_t stream) {
-  auto kern = fp8q::gemm_fp8_blockscaled_kernel<kPair, PROMOTE, ROW_B, GROUPED, OUT_BF16>;
-  static std::atomic<int> max_units[64];  // per instantiation, per device: co-resident clusters
-  const int smem = static_cast<int>(Cfg::smem_bytes);
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8Q_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = Cfg::kCG;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(fp8q::kGemmThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int units = max_units[dev].load(std::memory_order_acquire);
-  if (units == 0) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return FP8Q_ERR_CUDA;
+struct GemmLauncher {
+  static constexpr auto kern = fp8q::gemm_fp8_blockscaled_kernel<kPair, PROMOTE, ROW_B, GROUPED, OUT_BF16>;
+
+  static void config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, cudaStream_t stream) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = Cfg::kCG;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(fp8q::kGemmThreads);
+    cfg.dynamicSmemBytes = Cfg::smem_bytes;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+
+  // Co-resident units (CTAs, or CTA pairs) on the current device; sets the kernel's
+  // attributes on first use.  0 on failure.
+  static int max_units() {
+    static std::atomic<int> cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    int units = cached[dev].load(std::memory_order_acquire);
+    if (units) return units;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(Cfg::smem_bytes)) != cudaSuccess)
+      return 0;
     if (Cfg::kCG > 1 &&
         cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess)
-      return FP8Q_ERR_CUDA;
+      return 0;
     int sms = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return FP8Q_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    config(cfg, attr, nullptr);
     cfg.gridDim = dim3(static_cast<unsigned>(sms / Cfg::kCG * Cfg::kCG));
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0)
-      n = sms / Cfg::kCG;
-    units = n;
-    max_units[dev].store(units, std::memory_order_release);
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) n = sms / Cfg::kCG;
+    cached[dev].store(n, std::memory_order_release);
+    return n;
   }
-  const int64_t grid_units = work_units < units ? work_units : units;
-  if (grid_units <= 0) return FP8Q_OK;
-  cfg.gridDim = dim3(static_cast<unsigned>(grid_units * Cfg::kCG));
-  if (cudaLaunchKernelEx(&cfg, kern, tmA, tmB, args) != cudaSuccess) return FP8Q_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+
+  static int launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& args,
+                    int64_t grid_units, cudaStream_t stream) {
+    if (grid_units <= 0) return FP8Q_OK;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    config(cfg, attr, stream);
+    cfg.gridDim = dim3(static_cast<unsigned>(grid_units * Cfg::kCG));
+    if (cudaLaunchKernelEx(&cfg, kern, tmA, tmB, args) != cudaSuccess) return FP8Q_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+  }
+};
+
+// Work split of a dense GEMM over `units` co-resident CTAs: whole tiles in full waves,
+// and, when the last wave would leave most CTAs idle, its R tiles split into S K-chunks
+// (S = min(units / R, G / 2) >= 2) whose partials need a workspace of R*S tiles.
+struct SplitPlan {
+  int64_t tiles_full, tail_tiles, tail_split, grid_units;
+  size_t ws_bytes;
+};
+
+SplitPlan plan_split(int64_t tiles, int64_t G, int64_t units) {
+  SplitPlan sp{tiles, 0, 1, tiles < units ? tiles : units, 0};
+  if (kPair || units <= 0) return sp;
+  const int64_t full_waves = tiles / units, tail = tiles % units;
+  if (tail == 0) return sp;
+  int64_t split = units / tail;
+  if (split > G / 2) split = G / 2;
+  if (split < 2) return sp;
+  sp.tiles_full = full_waves * units;
+  sp.tail_tiles = tail;
+  sp.tail_split = split;
+  sp.grid_units = full_waves > 0 ? units : tail * split;
+  sp.ws_bytes = static_cast<size_t>(tail * split) * Cfg::kTileM * fp8q::kBN * sizeof(float);
+  return sp;
 }
 
 int check_gemm_common(const uint8_t* A, const uint8_t* B, const void* C, int out_dtype,
@@ -120,15 +155,46 @@ int check_gemm_common(const uint8_t* A, const uint8_t* B, const void* C, int out
   return FP8Q_OK;
 }
 
+// Launch one GEMM instantiation.  work: tiles (a bound for grouped).  Dense GEMMs given a
+// large enough workspace split their last partial wave along K and finish with a
+// reduction launch on the same stream.
+template <bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16>
+int run_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, GemmArgs a, int64_t work,
+             void* ws, size_t ws_bytes, cudaStream_t st) {
+  using L = GemmLauncher<PROMOTE, ROW_B, GROUPED, OUT_BF16>;
+  const int units = L::max_units();
+  if (units <= 0) return FP8Q_ERR_CUDA;
+  a.ws = nullptr;
+  a.tiles_full = static_cast<int>(work);
+  a.tail_tiles = 0;
+  a.tail_split = 1;
+  int64_t grid = work < units ? work : units;
+  if (!GROUPED && PROMOTE && ws != nullptr) {
+    const SplitPlan sp = plan_split(work, a.G, units);
+    if (sp.tail_tiles > 0 && sp.ws_bytes <= ws_bytes) {
+      a.ws = static_cast<float*>(ws);
+      a.tiles_full = static_cast<int>(sp.tiles_full);
+      a.tail_tiles = static_cast<int>(sp.tail_tiles);
+      a.tail_split = static_cast<int>(sp.tail_split);
+      grid = sp.grid_units;
+    }
+  }
+  int st_code = L::launch(tmA, tmB, a, grid, st);
+  if (st_code != FP8Q_OK || a.tail_tiles == 0) return st_code;
+  const int mt_total = static_cast<int>((a.M + Cfg::kTileM - 1) / Cfg::kTileM);
+  fp8q::splitk_reduce_kernel<OUT_BF16><<<a.tail_tiles * 128, 256, 0, st>>>(a, mt_total);
+  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
 template <bool PROMOTE, bool GROUPED>
 int dispatch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
-                  bool row_b, bool bf16, int64_t units, cudaStream_t st) {
+                  bool row_b, bool bf16, int64_t work, void* ws, size_t ws_bytes, cudaStream_t st) {
   if (row_b) {
-    return bf16 ? launch_gemm<PROMOTE, true, GROUPED, true>(tmA, tmB, a, units, st)
-                : launch_gemm<PROMOTE, true, GROUPED, false>(tmA, tmB, a, units, st);
+    return bf16 ? run_gemm<PROMOTE, true, GROUPED, true>(tmA, tmB, a, work, ws, ws_bytes, st)
+                : run_gemm<PROMOTE, true, GROUPED, false>(tmA, tmB, a, work, ws, ws_bytes, st);
   }
-  return bf16 ? launch_gemm<PROMOTE, false, GROUPED, true>(tmA, tmB, a, units, st)
-              : launch_gemm<PROMOTE, false, GROUPED, false>(tmA, tmB, a, units, st);
+  return bf16 ? run_gemm<PROMOTE, false, GROUPED, true>(tmA, tmB, a, work, ws, ws_bytes, st)
+              : run_gemm<PROMOTE, false, GROUPED, false>(tmA, tmB, a, work, ws, ws_bytes, st);
 }
 
 }  // namespace
@@ -221,10 +287,10 @@ int fp8q_quant_rowwise(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t
   return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
-int fp8_gemm_blockscaled(const uint8_t* A, const float* sA, int64_t ld_sa, const uint8_t* B,
-                         const float* sB, int64_t ld_sb, int b_scale_mode, void* C, int out_dtype,
-                         int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
-                         void* stream) {
+int fp8_gemm_blockscaled_ws(const uint8_t* A, const float* sA, int64_t ld_sa, const uint8_t* B,
+                            const float* sB, int64_t ld_sb, int b_scale_mode, void* C, int out_dtype,
+                            int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
+                            void* workspace, size_t workspace_bytes, void* stream) {
   if (M == 0 && N >= 0 && K >= 0) return FP8Q_OK;
   int st = check_gemm_common(A, B, C, out_dtype, M, N, K, lda, ldb, ldc);
   if (st != FP8Q_OK) return st;
@@ -242,8 +308,31 @@ int fp8_gemm_blockscaled(const uint8_t* A, const float* sA, int64_t ld_sa, const
   a.M = M; a.N = N; a.G = static_cast<int>(K / 128); a.m_offsets = nullptr; a.num_experts = 0;
   const int64_t tiles = ((M + Cfg::kTileM - 1) / Cfg::kTileM) * ((N + fp8q::kBN - 1) / fp8q::kBN);
   if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
+  if (workspace != nullptr && !aligned(workspace, 16)) return FP8Q_ERR_ALIGN;
   return dispatch_gemm<true, false>(tmA, tmB, a, b_scale_mode == FP8Q_BSCALE_ROW1x128,
-                                    out_dtype == FP8Q_OUT_BF16, tiles, static_cast<cudaStream_t>(stream));
+                                    out_dtype == FP8Q_OUT_BF16, tiles, workspace, workspace_bytes,
+                                    static_cast<cudaStream_t>(stream));
+}
+
+int fp8_gemm_blockscaled(const uint8_t* A, const float* sA, int64_t ld_sa, const uint8_t* B,
+                         const float* sB, int64_t ld_sb, int b_scale_mode, void* C, int out_dtype,
+                         int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
+                         void* stream) {
+  return fp8_gemm_blockscaled_ws(A, sA, ld_sa, B, sB, ld_sb, b_scale_mode, C, out_dtype, M, N, K,
+                                 lda, ldb, ldc, nullptr, 0, stream);
+}
+
+int fp8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, size_t* bytes) {
+  if (!bytes) return FP8Q_ERR_NULL;
+  *bytes = 0;
+  if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_SHAPE;
+  if (M == 0 || N == 0 || K == 0) return FP8Q_OK;
+  if (K % 128 != 0 || N % 128 != 0) return FP8Q_ERR_SHAPE;
+  const int units = GemmLauncher<true, false, false, true>::max_units();
+  if (units <= 0) return FP8Q_ERR_CUDA;
+  const int64_t tiles = ((M + Cfg::kTileM - 1) / Cfg::kTileM) * ((N + fp8q::kBN - 1) / fp8q::kBN);
+  *bytes = plan_split(tiles, K / 128, units).ws_bytes;
+  return FP8Q_OK;
 }
 
 int fp8_gemm_grouped(const uint8_t* A, const float* sA, int64_t ld_sa, const uint8_t* W,
@@ -270,7 +359,7 @@ int fp8_gemm_grouped(const uint8_t* A, const float* sA, int64_t ld_sa, const uin
   const int64_t nt = (N + fp8q::kBN - 1) / fp8q::kBN;
   const int64_t bound = ((max_sum_M + Cfg::kTileM - 1) / Cfg::kTileM + num_groups) * nt;
   if (bound > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  return dispatch_gemm<true, true>(tmA, tmB, a, false, out_dtype == FP8Q_OUT_BF16, bound,
+  return dispatch_gemm<true, true>(tmA, tmB, a, false, out_dtype == FP8Q_OUT_BF16, bound, nullptr, 0,
                                    static_cast<cudaStream_t>(stream));
 }
 
@@ -290,7 +379,8 @@ int fp8_gemm_nopromo(const uint8_t* A, const float* sA, const uint8_t* B, const 
   a.M = M; a.N = N; a.G = static_cast<int>(K / 128); a.m_offsets = nullptr; a.num_experts = 0;
   const int64_t tiles = ((M + Cfg::kTileM - 1) / Cfg::kTileM) * ((N + fp8q::kBN - 1) / fp8q::kBN);
   if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  return launch_gemm<false, false, false, false>(tmA, tmB, a, tiles, static_cast<cudaStream_t>(stream));
+  return run_gemm<false, false, false, false>(tmA, tmB, a, tiles, nullptr, 0,
+                                              static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -83,7 +83,48 @@ struct GemmArgs {
   int G;                // K / 128
   const int32_t* m_offsets;  // grouped: [E + 1] on the device
   int num_experts;
+  // Split-K of the last partial wave (dense only).  Tiles [0, tiles_full) are computed
+  // whole; the remaining tail_tiles are split into tail_split K-chunks, one per CTA of
+  // the last wave, whose FP32 partial tiles go to ws and are summed by
+  // splitk_reduce_kernel.  tail_tiles == 0: no split, ws unused.
+  float* ws;
+  int tiles_full;
+  int tail_tiles;
+  int tail_split;
 };
+
+// A unit of work of one CTA (or CTA pair): a tile and a range of its K-groups, written
+// to C (ws_index < 0) or as a partial tile to the workspace.
+struct Unit {
+  int tile, g0, g1, ws_index;
+};
+
+__device__ __forceinline__ int units_of(const GemmArgs& p, int num_tiles, int unit0, int units) {
+  if (p.tail_tiles == 0) return unit0 < num_tiles ? (num_tiles - unit0 + units - 1) / units : 0;
+  int n = unit0 < p.tiles_full ? (p.tiles_full - unit0 + units - 1) / units : 0;
+  if (unit0 < p.tail_tiles * p.tail_split) ++n;
+  return n;
+}
+
+__device__ __forceinline__ Unit unit_at(int i, const GemmArgs& p, int unit0, int units, int G) {
+  Unit u;
+  const int n_whole = p.tail_tiles == 0
+                          ? 0x7FFFFFFF
+                          : (unit0 < p.tiles_full ? (p.tiles_full - unit0 + units - 1) / units : 0);
+  if (i < n_whole) {
+    u.tile = unit0 + i * units;
+    u.g0 = 0;
+    u.g1 = G;
+    u.ws_index = -1;
+  } else {
+    const int r = unit0 / p.tail_split, ch = unit0 % p.tail_split;
+    u.tile = p.tiles_full + r;
+    u.g0 = static_cast<int>(static_cast<int64_t>(G) * ch / p.tail_split);
+    u.g1 = static_cast<int>(static_cast<int64_t>(G) * (ch + 1) / p.tail_split);
+    u.ws_index = unit0;
+  }
+  return u;
+}
 
 constexpr uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
@@ -256,6 +297,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (PAIR) cluster_sync();       // the peer's barriers are initialised before any remote use
   tc_fence_after();
   if (GROUPED) num_tiles = sched[p.num_experts];
+  const int n_units = units_of(p, num_tiles, unit0, units);
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp < kEpiWarp0) {
@@ -265,11 +307,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (lane == 0) {
         uint32_t it = 0;
         bool ok = true;
-        for (int t = unit0; ok && t < num_tiles; t += units) {
-          const Tile tl = decode_tile<GROUPED, Cfg::kTileM>(t, p, mt_total, nt_total, sched);
+        for (int ui = 0; ok && ui < n_units; ++ui) {
+          const Unit u = unit_at(ui, p, unit0, units, G);
+          const Tile tl = decode_tile<GROUPED, Cfg::kTileM>(u.tile, p, mt_total, nt_total, sched);
           const int32_t arow = static_cast<int32_t>(tl.row0 + 128 * rank);
           const int32_t brow = static_cast<int32_t>(tl.brow0 + Cfg::kBRows * rank);
-          for (int g = 0; g < G; ++g, ++it) {
+          for (int g = u.g0; g < u.g1; ++g, ++it) {
             const int s = it % S;
             const uint32_t ph = (it / S) & 1u;
             if (!mbar_wait(empty_bar(s), ph ^ 1u, kSiteProducer, abort_flag)) { ok = false; break; }
@@ -302,10 +345,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         constexpr uint32_t idesc = idesc_e4m3_f32(Cfg::kTileM, kBN);
         uint32_t it = 0, acc_it = 0;
         bool ok = true;
-        for (int t = unit0; ok && t < num_tiles; t += units) {
+        for (int ui = 0; ok && ui < n_units; ++ui) {
+          const Unit u = unit_at(ui, p, unit0, units, G);
           uint32_t buf = 0;
-          for (int g = 0; g < G; ++g, ++it) {
-            if (PROMOTE || g == 0) {
+          for (int g = u.g0; g < u.g1; ++g, ++it) {
+            if (PROMOTE || g == u.g0) {
               buf = acc_it & 1u;
               if (!mbar_wait(tempty_bar(buf), ((acc_it >> 1) & 1u) ^ 1u, kSiteMmaEmpty, abort_flag)) {
                 ok = false;
@@ -323,12 +367,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t b_addr = sbase + Cfg::b + s * Cfg::kBBytes;
 #pragma unroll
             for (int kk = 0; kk < kBK / 32; ++kk) {
-              const uint32_t accumulate = PROMOTE ? (kk > 0) : (g > 0 || kk > 0);
+              const uint32_t accumulate = PROMOTE ? (kk > 0) : (g > u.g0 || kk > 0);
               mma_f8<CG>(d, smem_desc_k_sw128(a_addr + 32 * kk), smem_desc_k_sw128(b_addr + 32 * kk),
                          idesc, accumulate);
             }
             if (PAIR) mma_commit_pair(empty_bar(s), 0x3); else mma_commit<1>(empty_bar(s));
-            if (PROMOTE || g == G - 1) {
+            if (PROMOTE || g == u.g1 - 1) {
               if (PAIR) mma_commit_pair(tfull_bar(buf), 0x3); else mma_commit<1>(tfull_bar(buf));
               ++acc_it;
             }
@@ -344,12 +388,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // 256 column scales (ROW mode) or, for 128x128 weight blocks, the two blocks'.
       uint32_t it = 0;
       bool ok = true;
-      for (int t = unit0; ok && t < num_tiles; t += units) {
-        const Tile tl = decode_tile<GROUPED, Cfg::kTileM>(t, p, mt_total, nt_total, sched);
+      for (int ui = 0; ok && ui < n_units; ++ui) {
+        const Unit u = unit_at(ui, p, unit0, units, G);
+        const Tile tl = decode_tile<GROUPED, Cfg::kTileM>(u.tile, p, mt_total, nt_total, sched);
         const int64_t r0 = tl.row0 + 128 * rank;
         const float* sB_tile =
             ROW_B ? nullptr : p.sB + (static_cast<int64_t>(tl.expert) * (p.N / 128) + tl.col0 / 128) * G;
-        for (int g = 0; g < G; ++g, ++it) {
+        for (int g = u.g0; g < u.g1; ++g, ++it) {
           const int r = it % R;
           if (!mbar_wait(sempty_bar(r), ((it / R) & 1u) ^ 1u, kSiteScales, abort_flag)) {
             ok = false;
@@ -403,8 +448,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // column set reaches the same named barriers.
     uint32_t acc_it = 0;
     bool ok = true;
-    for (int t = unit0; t < num_tiles; t += units) {
-      const Tile tl = decode_tile<GROUPED, Cfg::kTileM>(t, p, mt_total, nt_total, sched);
+    for (int ui = 0; ui < n_units; ++ui) {
+      const Unit u = unit_at(ui, p, unit0, units, G);
+      const Tile tl = decode_tile<GROUPED, Cfg::kTileM>(u.tile, p, mt_total, nt_total, sched);
       const int64_t m = tl.row0 + row_in_tile;
       const bool row_ok = m < tl.row_end;
       const int64_t n0 = tl.col0 + set * 128;
@@ -416,7 +462,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int j = 0; j < 64; ++j) acc[j] = make_float2(0.0f, 0.0f);
 
       if (PROMOTE) {
-        for (int g = 0; g < G; ++g) {
+        for (int g = u.g0; g < u.g1; ++g) {
           // This group's scales, staged by the scale producer (the ring advances with
           // every group of every tile, in the same order as acc_it).
           const int r = acc_it % R;
@@ -491,7 +537,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
 
       // ---- store the tile's rows: this thread owns row m, columns n0 .. n0+127
-      if (ok && row_ok && cols_ok) {
+      if (ok && u.ws_index >= 0) {
+        // split-K partial: the whole tile row (zeros outside C), summed later in fixed order
+        float* wrow = p.ws + (static_cast<int64_t>(u.ws_index) * Cfg::kTileM + row_in_tile) * kBN + set * 128;
+#pragma unroll
+        for (int j = 0; j < 64; j += 2)
+          *reinterpret_cast<float4*>(wrow + 2 * j) =
+              make_float4(acc[j].x, acc[j].y, acc[j + 1].x, acc[j + 1].y);
+      } else if (ok && row_ok && cols_ok) {
         if (OUT_BF16) {
           __nv_bfloat16* crow = reinterpret_cast<__nv_bfloat16*>(p.C) + m * p.ldc + n0;
 #pragma unroll
@@ -540,6 +593,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (PAIR) {
     __syncwarp();
     cluster_sync();               // neither CTA exits while its peer may still address it
+  }
+}
+
+// Sum of the split-K partial tiles of the last wave, in chunk order, written to C.
+// Grid: tail_tiles * 128 blocks (one tile row each) of 256 threads (one column each).
+template <bool OUT_BF16>
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const GemmArgs p, int mt_total) {
+  const int r = blockIdx.x / 128, row = blockIdx.x % 128, col = threadIdx.x;
+  const int t = p.tiles_full + r;
+  const int64_t m = static_cast<int64_t>(t % mt_total) * 128 + row;
+  const int64_t n = static_cast<int64_t>(t / mt_total) * kBN + col;
+  const float* w = p.ws + (static_cast<int64_t>(r) * p.tail_split * 128 + row) * kBN + col;
+  float acc = 0.0f;
+  for (int c = 0; c < p.tail_split; ++c) acc += w[static_cast<int64_t>(c) * 128 * kBN];
+  if (m < p.M && n < p.N) {
+    if (OUT_BF16)
+      reinterpret_cast<__nv_bfloat16*>(p.C)[m * p.ldc + n] = __float2bfloat16_rn(acc);
+    else
+      reinterpret_cast<float*>(p.C)[m * p.ldc + n] = acc;
   }
 }
 

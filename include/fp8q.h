@@ -31,6 +31,7 @@
 #ifndef FP8Q_H
 #define FP8Q_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -112,6 +113,31 @@ int fp8_gemm_blockscaled(const uint8_t* A, const float* sA, int64_t ld_sa, const
                          const float* sB, int64_t ld_sb, int b_scale_mode, void* C, int out_dtype,
                          int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
                          void* stream);
+
+/*
+ * Bytes of device workspace that fp8_gemm_blockscaled_ws can use for an M x N x K problem
+ * on the current device (0 when splitting the last wave would not help).  *bytes is set
+ * on success; K % 128 and N % 128 must be 0.
+ */
+int fp8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, size_t* bytes);
+
+/*
+ * fp8_gemm_blockscaled with a caller-owned device workspace (16-byte aligned).
+ *
+ * When the output tiles do not fill the last wave of SMs, the tiles of that wave are split
+ * along K (each chunk a whole number of 128-element groups, still promoted per group) over
+ * the otherwise idle SMs; each chunk's FP32 partial tile goes to the workspace and a second
+ * launch on the same stream adds the chunks in a fixed order and writes C.  Results are
+ * deterministic and within the same acceptance band as the unsplit order.  With
+ * workspace == NULL or workspace_bytes below fp8_gemm_workspace_size() the call computes
+ * without a split (exactly fp8_gemm_blockscaled).  The workspace is scratch: its contents
+ * are undefined afterwards, and calls that may run concurrently need distinct workspaces.
+ */
+int fp8_gemm_blockscaled_ws(const uint8_t* A, const float* sA, int64_t ld_sa, const uint8_t* B,
+                            const float* sB, int64_t ld_sb, int b_scale_mode, void* C,
+                            int out_dtype, int64_t M, int64_t N, int64_t K, int64_t lda,
+                            int64_t ldb, int64_t ldc, void* workspace, size_t workspace_bytes,
+                            void* stream);
 
 /*
  * Grouped (MoE expert) block-scaled GEMM [MoE]: rows m_offsets[e] .. m_offsets[e+1]-1 of A

@@ -86,6 +86,33 @@ def test_ragged_shapes(fq, M, N, K, out_fp32):
     _dense_case(fq, a, b, False, False, out_fp32, name=f"ragged {M}x{N}x{K}")
 
 
+@pytest.mark.parametrize("M,N,K,rowwise", [(128, 256, 512, False), (300, 1280, 1024, False),
+                                           (4096, 7168, 1024, False), (2048, 1024, 2048, True)])
+def test_split_last_wave_matches_unsplit(fq, M, N, K, rowwise):
+    """With a workspace the last partial wave is split along K; the result is deterministic
+    and inside the band of the unsplit result (and both inside the oracle's band)."""
+    import torch
+    rng = np.random.default_rng(M + N + K)
+    a = workloads.normal_bf16(rng, (M, K), 1.0, 0.001)
+    b = workloads.normal_bf16(rng, (N, K), 0.02 if not rowwise else 1.0)
+    qa, sa = fq.quant_act_1x128(to_dev_bf16(a), False)
+    qb, sb = (fq.quant_act_1x128(to_dev_bf16(b), False) if rowwise
+              else fq.quant_weight_128x128(to_dev_bf16(b), False))
+    assert fq.workspace_bytes(M, N, K) > 0
+    C1 = fq.gemm_blockscaled(qa, sa, qb, sb, out_dtype=torch.float32, b_rowwise=rowwise, split_k=True)
+    C1b = fq.gemm_blockscaled(qa, sa, qb, sb, out_dtype=torch.float32, b_rowwise=rowwise, split_k=True)
+    C0 = fq.gemm_blockscaled(qa, sa, qb, sb, out_dtype=torch.float32, b_rowwise=rowwise, split_k=False)
+    torch.cuda.synchronize()
+    assert fq.device_error() == 0
+    assert torch.equal(C1, C1b), "split result is deterministic"
+    rows = np.unique(np.concatenate([np.arange(0, M, max(1, M // 48)), [M - 1]]))
+    qa_r, sa_r = oracle.quant_act_1x128(a[rows], False)
+    qb_r, sb_r = oracle.quant_act_1x128(b, False) if rowwise else oracle.quant_weight_128x128(b, False)
+    C_ref, T = oracle.gemm_blockscaled_ref(qa_r, sa_r, qb_r, sb_r, rowwise)
+    assert_gemm_close("split", host(C1)[rows], C_ref, T, bf16=False)
+    assert_gemm_close("unsplit", host(C0)[rows], C_ref, T, bf16=False)
+
+
 @pytest.mark.parametrize("M,N,K", [(77, 256, 512), (128, 384, 256)])
 def test_rowwise_b_scales(fq, M, N, K):
     rng = np.random.default_rng(M * N)
