@@ -39,6 +39,8 @@ SIGNATURES = {
     "fp8_gemm_blockscaled_ws": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _i32, _vp, _i32,
                                        _i64, _i64, _i64, _i64, _i64, _i64, _vp, ctypes.c_size_t, _vp]),
     "fp8_gemm_workspace_size": (_i32, [_i64, _i64, _i64, ctypes.POINTER(ctypes.c_size_t)]),
+    "fp8_gemm_blockscaled_noalloc": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _i32, _vp, _i32,
+                                            _i64, _i64, _i64, _i64, _i64, _i64, _vp]),
     "fp8_gemm_grouped": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _i32, _vp, _i32,
                                 _i64, _i64, _i64, _vp]),
     "fp8_gemm_nopromo": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _vp]),

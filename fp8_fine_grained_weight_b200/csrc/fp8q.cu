@@ -199,6 +199,40 @@ int dispatch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs
 
 }  // namespace
 
+// ---------------------------------------------------------------------------------------
+// Fixed scratch for fp8_gemm_blockscaled_noalloc.
+//
+// Some callers cannot allocate device memory at the moment they run a GEMM: code that
+// runs under a memory budget fixed in advance (a pre-sized arena), allocator hooks or
+// callbacks that must not re-enter the allocator, or runtimes that forbid cudaMalloc
+// on their hot path.  For them the split-K workspace lives in this file-scope device
+// array instead of a caller buffer.  It is sized for the largest split plan on a 148-SM
+// B200 (at most one 128 x 256 FP32 partial tile per SM), and every GPU that loads this
+// library keeps it for the life of the process.
+constexpr size_t kStaticScratchBytes = size_t(20) << 20;   // 20 MiB
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+namespace {
+
+// Device address of g_static_scratch on the current device.  On the host the array's
+// name only stands for the symbol, so it is looked up once per device (with that device
+// current) and cached.  nullptr on failure.
+void* static_scratch_address() {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
+}  // namespace
+
 extern "C" {
 
 int fp8q_abi_version(void) { return 1; }
@@ -381,6 +415,25 @@ int fp8_gemm_nopromo(const uint8_t* A, const float* sA, const uint8_t* B, const 
   if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   return run_gemm<false, false, false, false>(tmA, tmB, a, tiles, nullptr, 0,
                                               static_cast<cudaStream_t>(stream));
+}
+
+// The split-K GEMM with its workspace in the library's fixed device scratch (see
+// g_static_scratch above); allocates nothing.
+int fp8_gemm_blockscaled_noalloc(const uint8_t* A, const float* sA, int64_t ld_sa,
+                                 const uint8_t* B, const float* sB, int64_t ld_sb,
+                                 int b_scale_mode, void* C, int out_dtype, int64_t M, int64_t N,
+                                 int64_t K, int64_t lda, int64_t ldb, int64_t ldc, void* stream) {
+  if (M == 0 && N >= 0 && K >= 0) return FP8Q_OK;
+  size_t need = 0;
+  int st = fp8_gemm_workspace_size(M, N, K, &need);
+  if (st != FP8Q_OK) return st;
+  if (need > kStaticScratchBytes) return FP8Q_ERR_SHAPE;   // the plan would overflow the array
+  void* scratch = static_scratch_address();
+  if (scratch == nullptr) return FP8Q_ERR_CUDA;
+  // Nothing in the scratch has to start at zero: every partial tile the reduction reads
+  // is written earlier in the same call.
+  return fp8_gemm_blockscaled_ws(A, sA, ld_sa, B, sB, ld_sb, b_scale_mode, C, out_dtype, M, N, K,
+                                 lda, ldb, ldc, scratch, kStaticScratchBytes, stream);
 }
 
 }  // extern "C"

@@ -140,6 +140,30 @@ int fp8_gemm_blockscaled_ws(const uint8_t* A, const float* sA, int64_t ld_sa, co
                             void* stream);
 
 /*
+ * fp8_gemm_blockscaled_ws for callers that cannot allocate device memory when they run the
+ * GEMM -- code with a memory budget fixed in advance, allocator callbacks that must not
+ * re-enter the allocator, runtimes that forbid cudaMalloc on their hot path.  The pages
+ * have no counterpart to this entry point; it exists for such callers only.
+ *
+ * The split-K workspace is a fixed 20 MiB device array inside the library (enough for
+ * every split plan on a 148-SM B200), held by every GPU that loads the library until the
+ * process exits.  The call allocates and frees nothing.  The caller passes inputs and
+ * outputs exactly as for fp8_gemm_blockscaled.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call before any
+ *    stream capture.
+ *  - Returns FP8Q_ERR_SHAPE when the problem's split would need more than 20 MiB
+ *    (possible only on a GPU with more SMs), besides the errors of fp8_gemm_blockscaled.
+ *  - All calls share the one array, which keeps the previous call's contents (nothing in
+ *    it needs to start at zero).  Calls that can overlap on the GPU -- on different
+ *    streams, or from different threads -- race on it and must be serialized by the caller.
+ */
+int fp8_gemm_blockscaled_noalloc(const uint8_t* A, const float* sA, int64_t ld_sa,
+                                 const uint8_t* B, const float* sB, int64_t ld_sb,
+                                 int b_scale_mode, void* C, int out_dtype, int64_t M, int64_t N,
+                                 int64_t K, int64_t lda, int64_t ldb, int64_t ldc, void* stream);
+
+/*
  * Grouped (MoE expert) block-scaled GEMM [MoE]: rows m_offsets[e] .. m_offsets[e+1]-1 of A
  * are multiplied by expert e's weights:
  *   C[m, :] = A[m, :] W[e]^T with the scaling of fp8_gemm_blockscaled (BLOCK mode).
