@@ -291,10 +291,14 @@ def run_gpu(args, rank, world):
 
 # ------------------------------------------------------------------------------ other workloads
 
-def _time_ms(fn, reps, flush_l2):
-    """Mean device time of fn() over reps, L2 flushed before each (outside the events)."""
+def _time_ms(fn, reps, flush_l2, warmup=2):
+    """Mean device time of fn() over reps, L2 flushed before each (outside the events).
+    Untimed warm-up calls first: a kernel variant's first launch pays one-time setup."""
     import torch
     stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
     tot = 0.0
     for _ in range(reps):
         flush_l2()

@@ -45,6 +45,7 @@ SIGNATURES = {
                                 _i64, _i64, _i64, _vp]),
     "fp8_gemm_nopromo": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _vp]),
     "fp8q_get_device_error": (_i32, [_vp]),
+    "fp8q_selftest_wait_timeout": (_i32, [ctypes.c_uint64, _vp]),
     "fp8q_status_string": (ctypes.c_char_p, [_i32]),
     "fp8q_abi_version": (_i32, []),
 }

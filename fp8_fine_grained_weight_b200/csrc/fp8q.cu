@@ -199,6 +199,19 @@ int dispatch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs
 
 }  // namespace
 
+namespace fp8q {
+// Self-test of the bounded wait: one thread waits on a barrier that nothing arrives on;
+// the wait gives up after timeout_ns and records (site 7 << 8) | FP8Q_ERR_TIMEOUT.
+__global__ void selftest_wait_kernel(uint64_t timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+    mbar_wait_ns(smem_u32(&bar), 0, 7, nullptr, timeout_ns);
+  }
+}
+}  // namespace fp8q
+
 // ---------------------------------------------------------------------------------------
 // Fixed scratch for fp8_gemm_blockscaled_noalloc.
 //
@@ -434,6 +447,15 @@ int fp8_gemm_blockscaled_noalloc(const uint8_t* A, const float* sA, int64_t ld_s
   // is written earlier in the same call.
   return fp8_gemm_blockscaled_ws(A, sA, ld_sa, B, sB, ld_sb, b_scale_mode, C, out_dtype, M, N, K,
                                  lda, ldb, ldc, scratch, kStaticScratchBytes, stream);
+}
+
+// Launches a one-thread kernel whose bounded wait cannot be satisfied; it returns after
+// timeout_ns with the timeout recorded in the device error word (read it with
+// fp8q_get_device_error).  Exercises the failure path without faulting the GPU.
+int fp8q_selftest_wait_timeout(uint64_t timeout_ns, void* stream) {
+  if (timeout_ns == 0 || timeout_ns > 1000000000ull) return FP8Q_ERR_SHAPE;
+  fp8q::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -199,9 +199,11 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& p, int mt_tot
     const int e = lo;
     int64_t r_begin, r_end;
     expert_rows(p, e, r_begin, r_end);
-    const int mte = static_cast<int>((r_end - r_begin + TILE_M - 1) / TILE_M);
+    // n-fastest inside an expert: concurrent tiles share a few row tiles of A and sweep
+    // the expert's weight columns, so A stays in L2 for large experts and the 1-2 row
+    // tiles of a small expert meet the same weight tile within one wave.
     const int local = t - sched[e];
-    const int mt = local % mte, nt = local / mte;
+    const int nt = local % nt_total, mt = local / nt_total;
     tl.row0 = r_begin + static_cast<int64_t>(mt) * TILE_M;
     tl.row_end = r_end;
     tl.col0 = static_cast<int64_t>(nt) * kBN;

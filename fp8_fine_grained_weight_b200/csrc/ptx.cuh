@@ -65,19 +65,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wait until the phase of parity `parity` has completed.  Returns false on timeout
 // (error recorded with `site`) or when `*abort` becomes nonzero.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned int site,
-                                          volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait_ns(uint32_t bar, uint32_t parity, unsigned int site,
+                                             volatile int* abort, uint64_t timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (abort != nullptr && *abort) return false;
-    if (globaltimer() - t0 > FP8Q_WAIT_TIMEOUT_NS) {
+    if (globaltimer() - t0 > timeout_ns) {
       record_error((site << 8) | 6u /* FP8Q_ERR_TIMEOUT */);
       if (abort != nullptr) *abort = 1;
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned int site,
+                                          volatile int* abort) {
+  return mbar_wait_ns(bar, parity, site, abort, FP8Q_WAIT_TIMEOUT_NS);
 }
 
 // ---------------------------------------------------------------- TMA

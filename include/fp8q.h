@@ -197,6 +197,12 @@ int fp8_gemm_nopromo(const uint8_t* A, const float* sA, const uint8_t* B, const 
  * device-side error was recorded, else (site << 8) | fp8q_status. */
 int fp8q_get_device_error(void* stream);
 
+/* Self-test of device-side failure detection: launches a one-thread kernel whose bounded
+ * wait on a barrier that nothing arrives on gives up after timeout_ns (1 ns .. 1 s) and
+ * records (7 << 8) | FP8Q_ERR_TIMEOUT in the device error word.  No fault, no hang: the
+ * context stays usable.  Returns FP8Q_ERR_SHAPE for an out-of-range timeout. */
+int fp8q_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
+
 /* Static description of a status code. */
 const char* fp8q_status_string(int status);
 
