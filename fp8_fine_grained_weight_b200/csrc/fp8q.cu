@@ -54,17 +54,24 @@ int encode_operand(CUtensorMap* tm, const void* base, uint64_t K, uint64_t rows,
   return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
-// The promoted GEMMs launch one CTA per 128 x 256 tile.  The CTA-pair variant
-// (cta_group::2, 256 x 256 tiles, half of B per CTA) is correct but slower here: with
-// promotion every 128 K the TMEM accumulator has to be released once per group, and
-// the pair turns that release into a cross-CTA round trip (about 0.5 us against a
-// 0.26 us group), which the two TMEM buffers cannot hide.
-constexpr bool kPair = false;
-using Cfg = fp8q::GemmCfg<kPair>;
+// Tile shapes.  Promotion every 128 K hands each TMEM accumulator from the tensor core to
+// the epilogue warps and back once per K-group.  The kernel template has two shapes:
+//  * single CTA, 128 x 256 tiles: 2 accumulator buffers of 256 columns;
+//  * CTA pair (cta_group::2), 256 x 128 tiles: 4 buffers of 128 columns per CTA, each CTA
+//    loading 128 rows of A and 64 of B per stage.
+// Both pass the same parity tests.  On B200 the pair is the slower of the two for every
+// promoted workload measured (dense 4096 x 7168 x 7168: 0.34 ms against 0.24 ms): its
+// groups are half as large, and the per-group cost of the hand-off (barrier waits, two
+// TMEM loads per epilogue warp, the release) is paid twice as often.  The launcher
+// therefore uses the single-CTA tiles; the pair instantiation is kept for the shapes
+// where that balance changes.
+bool dense_pair(int64_t) { return false; }
+bool grouped_pair(int64_t, int) { return false; }
 
-template <bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16>
+template <bool PAIR, bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16>
 struct GemmLauncher {
-  static constexpr auto kern = fp8q::gemm_fp8_blockscaled_kernel<kPair, PROMOTE, ROW_B, GROUPED, OUT_BF16>;
+  using Cfg = fp8q::GemmCfg<PAIR>;
+  static constexpr auto kern = fp8q::gemm_fp8_blockscaled_kernel<PAIR, PROMOTE, ROW_B, GROUPED, OUT_BF16>;
 
   static void config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, cudaStream_t stream) {
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -124,9 +131,11 @@ struct SplitPlan {
   size_t ws_bytes;
 };
 
+template <bool PAIR>
 SplitPlan plan_split(int64_t tiles, int64_t G, int64_t units) {
+  using Cfg = fp8q::GemmCfg<PAIR>;
   SplitPlan sp{tiles, 0, 1, tiles < units ? tiles : units, 0};
-  if (kPair || units <= 0) return sp;
+  if (units <= 0) return sp;
   const int64_t full_waves = tiles / units, tail = tiles % units;
   if (tail == 0) return sp;
   int64_t split = units / tail;
@@ -136,7 +145,7 @@ SplitPlan plan_split(int64_t tiles, int64_t G, int64_t units) {
   sp.tail_tiles = tail;
   sp.tail_split = split;
   sp.grid_units = full_waves > 0 ? units : tail * split;
-  sp.ws_bytes = static_cast<size_t>(tail * split) * Cfg::kTileM * fp8q::kBN * sizeof(float);
+  sp.ws_bytes = static_cast<size_t>(tail * split) * Cfg::kTileM * Cfg::kN * sizeof(float);
   return sp;
 }
 
@@ -158,10 +167,11 @@ int check_gemm_common(const uint8_t* A, const uint8_t* B, const void* C, int out
 // Launch one GEMM instantiation.  work: tiles (a bound for grouped).  Dense GEMMs given a
 // large enough workspace split their last partial wave along K and finish with a
 // reduction launch on the same stream.
-template <bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16>
+template <bool PAIR, bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16>
 int run_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, GemmArgs a, int64_t work,
              void* ws, size_t ws_bytes, cudaStream_t st) {
-  using L = GemmLauncher<PROMOTE, ROW_B, GROUPED, OUT_BF16>;
+  using L = GemmLauncher<PAIR, PROMOTE, ROW_B, GROUPED, OUT_BF16>;
+  using Cfg = fp8q::GemmCfg<PAIR>;
   const int units = L::max_units();
   if (units <= 0) return FP8Q_ERR_CUDA;
   a.ws = nullptr;
@@ -170,7 +180,7 @@ int run_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, GemmArgs a, int64_t
   a.tail_split = 1;
   int64_t grid = work < units ? work : units;
   if (!GROUPED && PROMOTE && ws != nullptr) {
-    const SplitPlan sp = plan_split(work, a.G, units);
+    const SplitPlan sp = plan_split<PAIR>(work, a.G, units);
     if (sp.tail_tiles > 0 && sp.ws_bytes <= ws_bytes) {
       a.ws = static_cast<float*>(ws);
       a.tiles_full = static_cast<int>(sp.tiles_full);
@@ -182,19 +192,27 @@ int run_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, GemmArgs a, int64_t
   int st_code = L::launch(tmA, tmB, a, grid, st);
   if (st_code != FP8Q_OK || a.tail_tiles == 0) return st_code;
   const int mt_total = static_cast<int>((a.M + Cfg::kTileM - 1) / Cfg::kTileM);
-  fp8q::splitk_reduce_kernel<OUT_BF16><<<a.tail_tiles * 128, 256, 0, st>>>(a, mt_total);
+  fp8q::splitk_reduce_kernel<OUT_BF16, Cfg::kTileM, Cfg::kN>
+      <<<a.tail_tiles * Cfg::kTileM, Cfg::kN, 0, st>>>(a, mt_total);
   return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
-template <bool PROMOTE, bool GROUPED>
-int dispatch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
-                  bool row_b, bool bf16, int64_t work, void* ws, size_t ws_bytes, cudaStream_t st) {
+// Promoted dense GEMM: tile shape, B scale mode and output type chosen at run time.
+template <bool PAIR>
+int dispatch_dense(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, bool row_b,
+                   bool bf16, int64_t work, void* ws, size_t ws_bytes, cudaStream_t st) {
   if (row_b) {
-    return bf16 ? run_gemm<PROMOTE, true, GROUPED, true>(tmA, tmB, a, work, ws, ws_bytes, st)
-                : run_gemm<PROMOTE, true, GROUPED, false>(tmA, tmB, a, work, ws, ws_bytes, st);
+    return bf16 ? run_gemm<PAIR, true, true, false, true>(tmA, tmB, a, work, ws, ws_bytes, st)
+                : run_gemm<PAIR, true, true, false, false>(tmA, tmB, a, work, ws, ws_bytes, st);
   }
-  return bf16 ? run_gemm<PROMOTE, false, GROUPED, true>(tmA, tmB, a, work, ws, ws_bytes, st)
-              : run_gemm<PROMOTE, false, GROUPED, false>(tmA, tmB, a, work, ws, ws_bytes, st);
+  return bf16 ? run_gemm<PAIR, true, false, false, true>(tmA, tmB, a, work, ws, ws_bytes, st)
+              : run_gemm<PAIR, true, false, false, false>(tmA, tmB, a, work, ws, ws_bytes, st);
+}
+
+template <bool PAIR>
+int64_t dense_tiles(int64_t M, int64_t N) {
+  using Cfg = fp8q::GemmCfg<PAIR>;
+  return ((M + Cfg::kTileM - 1) / Cfg::kTileM) * ((N + Cfg::kN - 1) / Cfg::kN);
 }
 
 }  // namespace
@@ -347,18 +365,21 @@ int fp8_gemm_blockscaled_ws(const uint8_t* A, const float* sA, int64_t ld_sa, co
   if (ld_sa < M) return FP8Q_ERR_SHAPE;
   if (b_scale_mode == FP8Q_BSCALE_ROW1x128 && ld_sb < N) return FP8Q_ERR_SHAPE;
   if (!aligned(sA, 4) || !aligned(sB, 4)) return FP8Q_ERR_ALIGN;
+  if (workspace != nullptr && !aligned(workspace, 16)) return FP8Q_ERR_ALIGN;
+  const bool pair = dense_pair(M);
   CUtensorMap tmA, tmB;
   if ((st = encode_operand(&tmA, A, K, M, lda, 128)) != FP8Q_OK) return st;
-  if ((st = encode_operand(&tmB, B, K, N, ldb, Cfg::kBRows)) != FP8Q_OK) return st;
+  const uint32_t b_rows = pair ? fp8q::GemmCfg<true>::kBRows : fp8q::GemmCfg<false>::kBRows;
+  if ((st = encode_operand(&tmB, B, K, N, ldb, b_rows)) != FP8Q_OK) return st;
   GemmArgs a{};
   a.sA = sA; a.ld_sa = ld_sa; a.sB = sB; a.ld_sb = ld_sb; a.C = C; a.ldc = ldc;
   a.M = M; a.N = N; a.G = static_cast<int>(K / 128); a.m_offsets = nullptr; a.num_experts = 0;
-  const int64_t tiles = ((M + Cfg::kTileM - 1) / Cfg::kTileM) * ((N + fp8q::kBN - 1) / fp8q::kBN);
+  const int64_t tiles = pair ? dense_tiles<true>(M, N) : dense_tiles<false>(M, N);
   if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  if (workspace != nullptr && !aligned(workspace, 16)) return FP8Q_ERR_ALIGN;
-  return dispatch_gemm<true, false>(tmA, tmB, a, b_scale_mode == FP8Q_BSCALE_ROW1x128,
-                                    out_dtype == FP8Q_OUT_BF16, tiles, workspace, workspace_bytes,
-                                    static_cast<cudaStream_t>(stream));
+  const bool row_b = b_scale_mode == FP8Q_BSCALE_ROW1x128, bf16 = out_dtype == FP8Q_OUT_BF16;
+  const auto s = static_cast<cudaStream_t>(stream);
+  return pair ? dispatch_dense<true>(tmA, tmB, a, row_b, bf16, tiles, workspace, workspace_bytes, s)
+              : dispatch_dense<false>(tmA, tmB, a, row_b, bf16, tiles, workspace, workspace_bytes, s);
 }
 
 int fp8_gemm_blockscaled(const uint8_t* A, const float* sA, int64_t ld_sa, const uint8_t* B,
@@ -375,10 +396,17 @@ int fp8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, size_t* bytes) {
   if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_SHAPE;
   if (M == 0 || N == 0 || K == 0) return FP8Q_OK;
   if (K % 128 != 0 || N % 128 != 0) return FP8Q_ERR_SHAPE;
-  const int units = GemmLauncher<true, false, false, true>::max_units();
-  if (units <= 0) return FP8Q_ERR_CUDA;
-  const int64_t tiles = ((M + Cfg::kTileM - 1) / Cfg::kTileM) * ((N + fp8q::kBN - 1) / fp8q::kBN);
-  *bytes = plan_split(tiles, K / 128, units).ws_bytes;
+  // The plan of the tile shape fp8_gemm_blockscaled_ws will choose for M; both B scale
+  // modes and output types share it.
+  if (dense_pair(M)) {
+    const int units = GemmLauncher<true, true, false, false, true>::max_units();
+    if (units <= 0) return FP8Q_ERR_CUDA;
+    *bytes = plan_split<true>(dense_tiles<true>(M, N), K / 128, units).ws_bytes;
+  } else {
+    const int units = GemmLauncher<false, true, false, false, true>::max_units();
+    if (units <= 0) return FP8Q_ERR_CUDA;
+    *bytes = plan_split<false>(dense_tiles<false>(M, N), K / 128, units).ws_bytes;
+  }
   return FP8Q_OK;
 }
 
@@ -394,20 +422,27 @@ int fp8_gemm_grouped(const uint8_t* A, const float* sA, int64_t ld_sa, const uin
   if (ld_sa < max_sum_M) return FP8Q_ERR_SHAPE;
   if (!aligned(sA, 4) || !aligned(sW, 4) || !aligned(m_offsets, 4)) return FP8Q_ERR_ALIGN;
   if (static_cast<int64_t>(num_groups) * N > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
+  const bool pair = grouped_pair(max_sum_M, num_groups);
   CUtensorMap tmA, tmB;
   if ((st = encode_operand(&tmA, A, K, max_sum_M, K, 128)) != FP8Q_OK) return st;
-  if ((st = encode_operand(&tmB, W, K, static_cast<uint64_t>(num_groups) * N, K, Cfg::kBRows)) != FP8Q_OK)
+  const uint32_t b_rows = pair ? fp8q::GemmCfg<true>::kBRows : fp8q::GemmCfg<false>::kBRows;
+  if ((st = encode_operand(&tmB, W, K, static_cast<uint64_t>(num_groups) * N, K, b_rows)) != FP8Q_OK)
     return st;
   GemmArgs a{};
   a.sA = sA; a.ld_sa = ld_sa; a.sB = sW; a.ld_sb = 0; a.C = C; a.ldc = N;
   a.M = max_sum_M; a.N = N; a.G = static_cast<int>(K / 128);
   a.m_offsets = m_offsets; a.num_experts = num_groups;
   // Upper bound on tiles (every group may add one partial m-tile) sizes the persistent grid.
-  const int64_t nt = (N + fp8q::kBN - 1) / fp8q::kBN;
-  const int64_t bound = ((max_sum_M + Cfg::kTileM - 1) / Cfg::kTileM + num_groups) * nt;
+  const int64_t tile_m = pair ? fp8q::GemmCfg<true>::kTileM : fp8q::GemmCfg<false>::kTileM;
+  const int64_t tile_n = pair ? fp8q::GemmCfg<true>::kN : fp8q::GemmCfg<false>::kN;
+  const int64_t bound = ((max_sum_M + tile_m - 1) / tile_m + num_groups) * ((N + tile_n - 1) / tile_n);
   if (bound > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  return dispatch_gemm<true, true>(tmA, tmB, a, false, out_dtype == FP8Q_OUT_BF16, bound, nullptr, 0,
-                                   static_cast<cudaStream_t>(stream));
+  const auto s = static_cast<cudaStream_t>(stream);
+  if (out_dtype == FP8Q_OUT_BF16)
+    return pair ? run_gemm<true, true, false, true, true>(tmA, tmB, a, bound, nullptr, 0, s)
+                : run_gemm<false, true, false, true, true>(tmA, tmB, a, bound, nullptr, 0, s);
+  return pair ? run_gemm<true, true, false, true, false>(tmA, tmB, a, bound, nullptr, 0, s)
+              : run_gemm<false, true, false, true, false>(tmA, tmB, a, bound, nullptr, 0, s);
 }
 
 int fp8_gemm_nopromo(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB, float* C,
@@ -420,14 +455,14 @@ int fp8_gemm_nopromo(const uint8_t* A, const float* sA, const uint8_t* B, const 
   if (!aligned(sA, 4) || !aligned(sB, 4)) return FP8Q_ERR_ALIGN;
   CUtensorMap tmA, tmB;
   if ((st = encode_operand(&tmA, A, K, M, lda, 128)) != FP8Q_OK) return st;
-  if ((st = encode_operand(&tmB, B, K, N, ldb, Cfg::kBRows)) != FP8Q_OK) return st;
+  if ((st = encode_operand(&tmB, B, K, N, ldb, fp8q::GemmCfg<false>::kBRows)) != FP8Q_OK) return st;
   GemmArgs a{};
   a.sA = sA; a.ld_sa = 0; a.sB = sB; a.ld_sb = 0; a.C = C; a.ldc = ldc;
   a.M = M; a.N = N; a.G = static_cast<int>(K / 128); a.m_offsets = nullptr; a.num_experts = 0;
-  const int64_t tiles = ((M + Cfg::kTileM - 1) / Cfg::kTileM) * ((N + fp8q::kBN - 1) / fp8q::kBN);
+  const int64_t tiles = dense_tiles<false>(M, N);
   if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  return run_gemm<false, false, false, false>(tmA, tmB, a, tiles, nullptr, 0,
-                                              static_cast<cudaStream_t>(stream));
+  return run_gemm<false, false, false, false, false>(tmA, tmB, a, tiles, nullptr, 0,
+                                                     static_cast<cudaStream_t>(stream));
 }
 
 // The split-K GEMM with its workspace in the library's fixed device scratch (see

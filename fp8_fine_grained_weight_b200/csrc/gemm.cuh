@@ -53,7 +53,7 @@
 
 namespace fp8q {
 
-constexpr int kBN = 256, kBK = 128;
+constexpr int kBK = 128;
 constexpr int kEpiWarps = 8;
 constexpr int kEpiWarp0 = 4;                      // first epilogue warp (second warpgroup)
 constexpr int kGemmThreads = 32 * (kEpiWarp0 + kEpiWarps);
@@ -131,9 +131,12 @@ constexpr uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a
 template <bool PAIR>
 struct GemmCfg {
   static constexpr int kCG = PAIR ? 2 : 1;              // CTAs per MMA
-  static constexpr int kStages = PAIR ? 6 : 4;
+  static constexpr int kN = PAIR ? 128 : 256;           // output columns per tile (MMA N)
+  static constexpr int kAccBufs = kTmemCols / kN;       // TMEM accumulator buffers
+  static constexpr int kSetCols = kN / 2;               // columns per epilogue column set
+  static constexpr int kStages = PAIR ? 8 : 4;
   static constexpr int kTileM = 128 * kCG;              // output rows per (pair) tile
-  static constexpr int kBRows = kBN / kCG;              // rows of B each CTA loads
+  static constexpr int kBRows = kN / kCG;               // rows of B each CTA loads
   static constexpr uint32_t kABytes = 128 * kBK;        // per CTA per stage
   static constexpr uint32_t kBBytes = kBRows * kBK;
   static constexpr uint32_t kStageTx = (kABytes + kBBytes) * kCG;  // bytes per full barrier phase
@@ -145,9 +148,9 @@ struct GemmCfg {
   static constexpr uint32_t b = a + kStages * kABytes;
   static constexpr uint32_t bars = b + kStages * kBBytes;
   static constexpr int kScaleSlots = 8;                  // scale ring depth (groups)
-  static constexpr uint32_t kSlotFloats = 128 + 256;     // A row scales + B scales
-  // full[S], empty[S], tfull[2], tempty[2], drain, sfull[R], sempty[R]
-  static constexpr uint32_t n_bars = 2 * kStages + 5 + 2 * kScaleSlots;
+  static constexpr uint32_t kSlotFloats = 128 + kN;      // A row scales + B scales
+  // full[S], empty[S], tfull[NB], tempty[NB], drain, sfull[R], sempty[R]
+  static constexpr uint32_t n_bars = 2 * kStages + 2 * kAccBufs + 1 + 2 * kScaleSlots;
   static constexpr uint32_t misc = align_up(bars + 8 * n_bars, 16);   // tmem slot, abort flag
   static constexpr uint32_t sched = align_up(misc + 16, 16);          // int[kMaxGroups + 1]
   static constexpr uint32_t sbrow = align_up(sched + 4 * (kMaxGroups + 1), 128);  // float[2][2][128]
@@ -156,7 +159,9 @@ struct GemmCfg {
   static constexpr uint32_t smem_bytes = end + 1024;                  // + base alignment slack
   static_assert(a % 1024 == 0 && b % 1024 == 0 && kABytes % 1024 == 0 && kBBytes % 1024 == 0,
                 "swizzle atoms");
-  static_assert(sbrow % 16 == 0 && sring % 16 == 0, "float4 reads of the scale slots");
+  static_assert(sbrow % 16 == 0 && sring % 16 == 0 && kSlotFloats % 4 == 0,
+                "float4 reads of the scale slots");
+  static_assert(kSetCols % 64 == 0 && kN % 128 == 0, "epilogue column sets of 64-column loads");
   static_assert(smem_bytes <= 232448, "fits the 227 KB opt-in shared memory");
 };
 
@@ -178,7 +183,7 @@ __device__ __forceinline__ void expert_rows(const GemmArgs& p, int e, int64_t& r
   r_end = en;
 }
 
-template <bool GROUPED, int TILE_M>
+template <bool GROUPED, int TILE_M, int TILE_N>
 __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& p, int mt_total, int nt_total,
                                             const int* sched) {
   Tile tl;
@@ -186,7 +191,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& p, int mt_tot
     const int mt = t % mt_total, nt = t / mt_total;
     tl.row0 = static_cast<int64_t>(mt) * TILE_M;
     tl.row_end = p.M;
-    tl.col0 = static_cast<int64_t>(nt) * kBN;
+    tl.col0 = static_cast<int64_t>(nt) * TILE_N;
     tl.brow0 = tl.col0;
     tl.expert = 0;
   } else {
@@ -206,7 +211,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& p, int mt_tot
     const int nt = local % nt_total, mt = local / nt_total;
     tl.row0 = r_begin + static_cast<int64_t>(mt) * TILE_M;
     tl.row_end = r_end;
-    tl.col0 = static_cast<int64_t>(nt) * kBN;
+    tl.col0 = static_cast<int64_t>(nt) * TILE_N;
     tl.brow0 = static_cast<int64_t>(e) * p.N + tl.col0;
     tl.expert = e;
   }
@@ -224,6 +229,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   using Cfg = GemmCfg<PAIR>;
   constexpr int CG = Cfg::kCG;
   constexpr int S = Cfg::kStages;
+  constexpr int NB = Cfg::kAccBufs;
+  constexpr int kN = Cfg::kN;
+  constexpr int kSetCols = Cfg::kSetCols;
+  static_assert(PROMOTE || !PAIR, "the no-promotion variant runs on single CTAs");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -232,11 +241,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
   auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * S + b); };
-  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * S + 2 + b); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * S + 4);
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * S + NB + b); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * S + 2 * NB);
   constexpr int R = Cfg::kScaleSlots;
-  auto sfull_bar = [&](int r) { return bar0 + 8u * (2 * S + 5 + r); };
-  auto sempty_bar = [&](int r) { return bar0 + 8u * (2 * S + 5 + R + r); };
+  auto sfull_bar = [&](int r) { return bar0 + 8u * (2 * S + 2 * NB + 1 + r); };
+  auto sempty_bar = [&](int r) { return bar0 + 8u * (2 * S + 2 * NB + 1 + R + r); };
   float* sring = reinterpret_cast<float*>(smem + Cfg::sring);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::misc + 4);
@@ -254,7 +263,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NB; ++b) {
       mbar_init(tfull_bar(b), 1);
       mbar_init(tempty_bar(b), Cfg::kTemptyArrivals);
     }
@@ -275,7 +284,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_relinquish<CG>();
   }
 
-  const int nt_total = static_cast<int>((p.N + kBN - 1) / kBN);
+  const int nt_total = static_cast<int>((p.N + kN - 1) / kN);
   int mt_total = 0, num_tiles = 0;
   if (!GROUPED) {
     mt_total = static_cast<int>((p.M + Cfg::kTileM - 1) / Cfg::kTileM);
@@ -311,7 +320,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         bool ok = true;
         for (int ui = 0; ok && ui < n_units; ++ui) {
           const Unit u = unit_at(ui, p, unit0, units, G);
-          const Tile tl = decode_tile<GROUPED, Cfg::kTileM>(u.tile, p, mt_total, nt_total, sched);
+          const Tile tl = decode_tile<GROUPED, Cfg::kTileM, Cfg::kN>(u.tile, p, mt_total, nt_total, sched);
           const int32_t arow = static_cast<int32_t>(tl.row0 + 128 * rank);
           const int32_t brow = static_cast<int32_t>(tl.brow0 + Cfg::kBRows * rank);
           for (int g = u.g0; g < u.g1; ++g, ++it) {
@@ -344,7 +353,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp == 1) {
       // ---------------------------------------------------------- MMA issuer
       if (lane == 0 && mma_cta) {
-        constexpr uint32_t idesc = idesc_e4m3_f32(Cfg::kTileM, kBN);
+        constexpr uint32_t idesc = idesc_e4m3_f32(Cfg::kTileM, kN);
         uint32_t it = 0, acc_it = 0;
         bool ok = true;
         for (int ui = 0; ok && ui < n_units; ++ui) {
@@ -352,8 +361,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint32_t buf = 0;
           for (int g = u.g0; g < u.g1; ++g, ++it) {
             if (PROMOTE || g == u.g0) {
-              buf = acc_it & 1u;
-              if (!mbar_wait(tempty_bar(buf), ((acc_it >> 1) & 1u) ^ 1u, kSiteMmaEmpty, abort_flag)) {
+              buf = acc_it % NB;
+              if (!mbar_wait(tempty_bar(buf), ((acc_it / NB) & 1u) ^ 1u, kSiteMmaEmpty, abort_flag)) {
                 ok = false;
                 break;
               }
@@ -364,7 +373,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               break;
             }
             tc_fence_after();
-            const uint32_t d = tmem_base + buf * kBN;
+            const uint32_t d = tmem_base + buf * kN;
             const uint32_t a_addr = sbase + Cfg::a + s * Cfg::kABytes;
             const uint32_t b_addr = sbase + Cfg::b + s * Cfg::kBBytes;
 #pragma unroll
@@ -386,13 +395,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     } else if (warp == 2 && PROMOTE) {
       // ---------------------------------------------------------- scale producer
-      // Slot layout: [0, 128) A scales of this CTA's 128 rows; [128, 384) B scales: the
-      // 256 column scales (ROW mode) or, for 128x128 weight blocks, the two blocks'.
+      // Slot layout: [0, 128) A scales of this CTA's 128 rows; [128, 128 + kN) B scales:
+      // the tile's kN column scales (ROW mode) or, for 128x128 weight blocks, the kN / 128
+      // blocks' scales.
       uint32_t it = 0;
       bool ok = true;
       for (int ui = 0; ok && ui < n_units; ++ui) {
         const Unit u = unit_at(ui, p, unit0, units, G);
-        const Tile tl = decode_tile<GROUPED, Cfg::kTileM>(u.tile, p, mt_total, nt_total, sched);
+        const Tile tl = decode_tile<GROUPED, Cfg::kTileM, Cfg::kN>(u.tile, p, mt_total, nt_total, sched);
         const int64_t r0 = tl.row0 + 128 * rank;
         const float* sB_tile =
             ROW_B ? nullptr : p.sB + (static_cast<int64_t>(tl.expert) * (p.N / 128) + tl.col0 / 128) * G;
@@ -412,11 +422,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (ROW_B) {
             const float* sb_g = p.sB + static_cast<int64_t>(g) * p.ld_sb;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < kN / 32; ++j) {
               const int64_t n = tl.col0 + 32 * j + lane;
               cp_async_4(slot + 4u * (128 + 32 * j + lane), sb_g + (n < p.N ? n : 0), n < p.N);
             }
-          } else if (lane < 2) {
+          } else if (lane < kN / 128) {
             const bool v = tl.col0 + 128 * lane < p.N;
             cp_async_4(slot + 4u * (128 + lane), sB_tile + (v ? lane * G + g : 0), v);
           }
@@ -448,20 +458,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // The epilogue never leaves its loops early: after an abort it keeps walking the
     // (uniform) tile/group structure without touching TMEM, so that every thread of a
     // column set reaches the same named barriers.
+    constexpr int kLoads = kSetCols / 64;   // 64-column TMEM loads per group
     uint32_t acc_it = 0;
     bool ok = true;
     for (int ui = 0; ui < n_units; ++ui) {
       const Unit u = unit_at(ui, p, unit0, units, G);
-      const Tile tl = decode_tile<GROUPED, Cfg::kTileM>(u.tile, p, mt_total, nt_total, sched);
+      const Tile tl = decode_tile<GROUPED, Cfg::kTileM, Cfg::kN>(u.tile, p, mt_total, nt_total, sched);
       const int64_t m = tl.row0 + row_in_tile;
       const bool row_ok = m < tl.row_end;
-      const int64_t n0 = tl.col0 + set * 128;
+      const int64_t n0 = tl.col0 + set * kSetCols;
       const bool cols_ok = n0 < p.N;
       // acc[i] holds columns 2i, 2i+1 of this thread's row (packed FP32 pairs: the
       // promotion runs on the f32x2 FMA path, two accumulations per instruction).
-      float2 acc[64];
+      float2 acc[kSetCols / 2];
 #pragma unroll
-      for (int j = 0; j < 64; ++j) acc[j] = make_float2(0.0f, 0.0f);
+      for (int j = 0; j < kSetCols / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
 
       if (PROMOTE) {
         for (int g = u.g0; g < u.g1; ++g) {
@@ -471,22 +482,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const float* slot = sring + Cfg::kSlotFloats * r;
           if (ok) ok = mbar_wait(sfull_bar(r), (acc_it / R) & 1u, kSiteScales, abort_flag);
           const float sa_cur = slot[quad * 32 + lane];
-          const float sb_cur = ROW_B ? 0.0f : slot[128 + set];
-          const float* sbv = slot + 128 + set * 128;        // ROW mode column scales
-          const uint32_t buf = acc_it & 1u;
-          if (ok) ok = mbar_wait(tfull_bar(buf), (acc_it >> 1) & 1u, kSiteEpilogue, abort_flag);
+          const float sb_cur = ROW_B ? 0.0f : slot[128 + set * kSetCols / 128];
+          const float* sbv = slot + 128 + set * kSetCols;   // ROW mode column scales
+          const uint32_t buf = acc_it % NB;
+          if (ok) ok = mbar_wait(tfull_bar(buf), (acc_it / NB) & 1u, kSiteEpilogue, abort_flag);
           if (ok) {
             tc_fence_after();
             const uint32_t taddr =
-                tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + buf * kBN + set * 128;
+                tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + buf * kN + set * kSetCols;
             const float2 sc2 = make_float2(sa_cur * sb_cur, sa_cur * sb_cur);
             const float2 sa2 = make_float2(sa_cur, sa_cur);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            for (int h = 0; h < kLoads; ++h) {
               uint32_t r[64];
               tmem_ld_64cols(taddr + h * 64, r);
               tmem_ld_wait();
-              if (h == 1) release(buf);   // TMEM buffer free for group g+2
+              if (h == kLoads - 1) release(buf);   // TMEM buffer free for group g + NB
 #pragma unroll
               for (int j = 0; j < 64; j += 4) {
                 const float2 p0 = make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
@@ -512,21 +523,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const float sa = row_ok ? __ldg(p.sA + m) : 0.0f;
         float* slot = sb_slots;
         named_bar_sync(1 + set, 128);   // previous tile's readers are done with the slot
-        slot[tid_in_set] = cols_ok ? __ldg(p.sB + n0 + tid_in_set) : 0.0f;
+        if (tid_in_set < kSetCols)
+          slot[tid_in_set] = cols_ok ? __ldg(p.sB + n0 + tid_in_set) : 0.0f;
         named_bar_sync(1 + set, 128);
-        const uint32_t buf = acc_it & 1u;
-        if (ok) ok = mbar_wait(tfull_bar(buf), (acc_it >> 1) & 1u, kSiteEpilogue, abort_flag);
+        const uint32_t buf = acc_it % NB;
+        if (ok) ok = mbar_wait(tfull_bar(buf), (acc_it / NB) & 1u, kSiteEpilogue, abort_flag);
         if (ok) {
           tc_fence_after();
           const uint32_t taddr =
-              tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + buf * kBN + set * 128;
+              tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + buf * kN + set * kSetCols;
           const float2 sa2 = make_float2(sa, sa);
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
+          for (int h = 0; h < kLoads; ++h) {
             uint32_t r[64];
             tmem_ld_64cols(taddr + h * 64, r);
             tmem_ld_wait();
-            if (h == 1) release(buf);
+            if (h == kLoads - 1) release(buf);
 #pragma unroll
             for (int j = 0; j < 64; j += 2) {
               const float2 pr = make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
@@ -538,19 +550,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         ++acc_it;
       }
 
-      // ---- store the tile's rows: this thread owns row m, columns n0 .. n0+127
+      // ---- store the tile's rows: this thread owns row m, columns n0 .. n0 + kSetCols
       if (ok && u.ws_index >= 0) {
         // split-K partial: the whole tile row (zeros outside C), summed later in fixed order
-        float* wrow = p.ws + (static_cast<int64_t>(u.ws_index) * Cfg::kTileM + row_in_tile) * kBN + set * 128;
+        float* wrow = p.ws + (static_cast<int64_t>(u.ws_index) * Cfg::kTileM + row_in_tile) * kN +
+                      set * kSetCols;
 #pragma unroll
-        for (int j = 0; j < 64; j += 2)
+        for (int j = 0; j < kSetCols / 2; j += 2)
           *reinterpret_cast<float4*>(wrow + 2 * j) =
               make_float4(acc[j].x, acc[j].y, acc[j + 1].x, acc[j + 1].y);
       } else if (ok && row_ok && cols_ok) {
         if (OUT_BF16) {
           __nv_bfloat16* crow = reinterpret_cast<__nv_bfloat16*>(p.C) + m * p.ldc + n0;
 #pragma unroll
-          for (int j = 0; j < 64; j += 4) {
+          for (int j = 0; j < kSetCols / 2; j += 4) {
             __nv_bfloat162 h0 = __float22bfloat162_rn(acc[j + 0]);
             __nv_bfloat162 h1 = __float22bfloat162_rn(acc[j + 1]);
             __nv_bfloat162 h2 = __float22bfloat162_rn(acc[j + 2]);
@@ -565,7 +578,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         } else {
           float* crow = reinterpret_cast<float*>(p.C) + m * p.ldc + n0;
 #pragma unroll
-          for (int j = 0; j < 64; j += 2)
+          for (int j = 0; j < kSetCols / 2; j += 2)
             *reinterpret_cast<float4*>(crow + 2 * j) =
                 make_float4(acc[j].x, acc[j].y, acc[j + 1].x, acc[j + 1].y);
         }
@@ -599,16 +612,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // Sum of the split-K partial tiles of the last wave, in chunk order, written to C.
-// Grid: tail_tiles * 128 blocks (one tile row each) of 256 threads (one column each).
-template <bool OUT_BF16>
-__global__ void __launch_bounds__(256) splitk_reduce_kernel(const GemmArgs p, int mt_total) {
-  const int r = blockIdx.x / 128, row = blockIdx.x % 128, col = threadIdx.x;
+// Grid: tail_tiles * TILE_M blocks (one tile row each) of TILE_N threads (one column each).
+template <bool OUT_BF16, int TILE_M, int TILE_N>
+__global__ void __launch_bounds__(TILE_N) splitk_reduce_kernel(const GemmArgs p, int mt_total) {
+  const int r = blockIdx.x / TILE_M, row = blockIdx.x % TILE_M, col = threadIdx.x;
   const int t = p.tiles_full + r;
-  const int64_t m = static_cast<int64_t>(t % mt_total) * 128 + row;
-  const int64_t n = static_cast<int64_t>(t / mt_total) * kBN + col;
-  const float* w = p.ws + (static_cast<int64_t>(r) * p.tail_split * 128 + row) * kBN + col;
+  const int64_t m = static_cast<int64_t>(t % mt_total) * TILE_M + row;
+  const int64_t n = static_cast<int64_t>(t / mt_total) * TILE_N + col;
+  const float* w = p.ws + (static_cast<int64_t>(r) * p.tail_split * TILE_M + row) * TILE_N + col;
   float acc = 0.0f;
-  for (int c = 0; c < p.tail_split; ++c) acc += w[static_cast<int64_t>(c) * 128 * kBN];
+  for (int c = 0; c < p.tail_split; ++c) acc += w[static_cast<int64_t>(c) * TILE_M * TILE_N];
   if (m < p.M && n < p.N) {
     if (OUT_BF16)
       reinterpret_cast<__nv_bfloat16*>(p.C)[m * p.ldc + n] = __float2bfloat16_rn(acc);

@@ -87,7 +87,7 @@ def test_ragged_shapes(fq, M, N, K, out_fp32):
 
 
 @pytest.mark.parametrize("M,N,K,rowwise", [(128, 256, 512, False), (300, 1280, 1024, False),
-                                           (4096, 7168, 1024, False), (2048, 1024, 2048, True)])
+                                           (4096, 7168, 1024, False), (2048, 512, 2048, True)])
 def test_split_last_wave_matches_unsplit(fq, M, N, K, rowwise):
     """With a workspace the last partial wave is split along K; the result is deterministic
     and inside the band of the unsplit result (and both inside the oracle's band)."""
@@ -166,7 +166,7 @@ def test_wgrad_full_size_sampled_rows(fq):
 # ------------------------------------------------------------------------------------ grouped
 
 def _grouped_case(fq, counts, N, K, pow2_a, out_fp32, a_std=1.0, b_std=0.006, rows=None,
-                  seed=0, bits=None, name="grouped"):
+                  seed=0, bits=None, name="grouped", alloc_rows=1):
     import torch
     counts = np.asarray(counts, dtype=np.int64)
     E = counts.size
@@ -174,17 +174,18 @@ def _grouped_case(fq, counts, N, K, pow2_a, out_fp32, a_std=1.0, b_std=0.006, ro
     M = int(off[-1])
     if bits is None:
         rng = np.random.default_rng(seed)
-        a_bits = workloads.normal_bf16(rng, (max(M, 1), K), a_std, 0.001)
+        a_bits = workloads.normal_bf16(rng, (max(M, alloc_rows), K), a_std, 0.001)
         w_bits = workloads.normal_bf16(rng, (E, N, K), b_std)
     else:
         a_bits, w_bits = bits
     qa, sa = fq.quant_act_1x128(to_dev_bf16(a_bits), pow2_a)
     qw, sw = fq.quant_weight_128x128(to_dev_bf16(w_bits), False)
     out_dtype = torch.float32 if out_fp32 else torch.bfloat16
-    C = torch.full((max(M, 1), N), float("nan"), dtype=out_dtype, device="cuda")
+    C = torch.full((max(M, alloc_rows), N), float("nan"), dtype=out_dtype, device="cuda")
     fq.gemm_grouped(qa, sa, qw, sw, to_dev(off), out_dtype=out_dtype, out=C)
     torch.cuda.synchronize()
     assert fq.device_error() == 0
+    assert torch.isnan(C[M:]).all(), "rows past the last offset are not written"
     if M == 0:
         return
     rows = np.arange(M) if rows is None else np.asarray(rows)
@@ -213,6 +214,14 @@ def _grouped_case(fq, counts, N, K, pow2_a, out_fp32, a_std=1.0, b_std=0.006, ro
 @pytest.mark.parametrize("out_fp32", [True, False])
 def test_grouped_small_with_empty_groups(fq, out_fp32):
     _grouped_case(fq, [0, 5, 130, 1, 0, 77, 256, 0], 256, 384, False, out_fp32, seed=1)
+
+
+@pytest.mark.parametrize("out_fp32", [True, False])
+def test_grouped_ragged_with_slack_rows(fq, out_fp32):
+    """Ragged experts (1..600 rows, some empty), N = 384, and an A allocation of 4096 rows
+    of which only the first 983 belong to experts: the slack rows stay unwritten."""
+    _grouped_case(fq, [0, 5, 300, 1, 0, 77, 600, 0], 384, 384, False, out_fp32, seed=5,
+                  alloc_rows=4096)
 
 
 def test_grouped_unwritten_rows_untouched(fq):
