@@ -26,7 +26,8 @@ OUT_BF16, OUT_FP32 = 0, 1
 BSCALE_BLOCK, BSCALE_ROW = 0, 1
 
 STATUS = {0: "FP8Q_OK", 1: "FP8Q_ERR_NULL", 2: "FP8Q_ERR_SHAPE", 3: "FP8Q_ERR_ALIGN",
-          4: "FP8Q_ERR_UNSUPPORTED", 5: "FP8Q_ERR_CUDA", 6: "FP8Q_ERR_TIMEOUT"}
+          4: "FP8Q_ERR_UNSUPPORTED", 5: "FP8Q_ERR_CUDA", 6: "FP8Q_ERR_TIMEOUT",
+          7: "FP8Q_ERR_SCALE"}
 
 # name -> (restype, argtypes); mirrors include/fp8q.h
 _i64, _i32, _vp, _f = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_float
@@ -36,6 +37,8 @@ SIGNATURES = {
     "fp8q_quant_rowwise": (_i32, [_vp, _i64, _i64, _i64, _vp, _i64, _vp, _i32, _vp]),
     "fp8_gemm_blockscaled": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _i32, _vp, _i32,
                                     _i64, _i64, _i64, _i64, _i64, _i64, _vp]),
+    "fp8_gemm_blockscaled_ue8m0": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _i32, _vp, _i32,
+                                          _i64, _i64, _i64, _i64, _i64, _i64, _vp]),
     "fp8_gemm_blockscaled_ws": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _i32, _vp, _i32,
                                        _i64, _i64, _i64, _i64, _i64, _i64, _vp, ctypes.c_size_t, _vp]),
     "fp8_gemm_workspace_size": (_i32, [_i64, _i64, _i64, ctypes.POINTER(ctypes.c_size_t)]),
@@ -218,6 +221,33 @@ def gemm_blockscaled(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: t
           sb.data_ptr(), sb.stride(0) if b_rowwise else 0,
           BSCALE_ROW if b_rowwise else BSCALE_BLOCK, out.data_ptr(), _out_code(out.dtype),
           M, N, K, qa.stride(0), qb.stride(0), out.stride(0), ws_ptr, ws_len, _stream(qa))
+    return out
+
+
+def gemm_blockscaled_ue8m0(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor,
+                           out_dtype=torch.bfloat16, b_rowwise: bool = False,
+                           out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """C = A B^T for power-of-two scales, scaled inside the tensor core (UE8M0 block scales).
+
+    Same operands as ``gemm_blockscaled``; every scale must be a power of two in
+    [2^-127, 2^127] (the quantizers' ``pow2`` option).  Other scales are reported through
+    ``device_error()`` as (8 << 8) | FP8Q_ERR_SCALE.
+    """
+    qa, qb = _u8(qa), _u8(qb)
+    _need(qa, torch.uint8, "qa", 2)
+    _need(qb, torch.uint8, "qb", 2)
+    _need(sa, torch.float32, "sa", 2)
+    _need(sb, torch.float32, "sb", 2)
+    M, K = qa.shape
+    N = qb.shape[0]
+    if qb.shape[1] != K:
+        raise ValueError("qa and qb disagree on K")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=qa.device)
+    _call("fp8_gemm_blockscaled_ue8m0", qa.data_ptr(), sa.data_ptr(), sa.stride(0), qb.data_ptr(),
+          sb.data_ptr(), sb.stride(0) if b_rowwise else 0,
+          BSCALE_ROW if b_rowwise else BSCALE_BLOCK, out.data_ptr(), _out_code(out.dtype),
+          M, N, K, qa.stride(0), qb.stride(0), out.stride(0), _stream(qa))
     return out
 
 

@@ -15,6 +15,7 @@
 
 #include "../../include/fp8q.h"
 #include "gemm.cuh"
+#include "gemm_ue8m0.cuh"
 #include "quant.cuh"
 
 namespace {
@@ -215,6 +216,37 @@ int64_t dense_tiles(int64_t M, int64_t N) {
   return ((M + Cfg::kTileM - 1) / Cfg::kTileM) * ((N + Cfg::kN - 1) / Cfg::kN);
 }
 
+static_assert(fp8q::kErrScale == FP8Q_ERR_SCALE, "device status code of a bad scale");
+
+// Launch of the power-of-two-scale GEMM: one persistent CTA per SM (kernel attributes set
+// and the co-resident count cached per device on first use).
+template <bool ROW_B, bool OUT_BF16>
+int run_gemm_ue8m0(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
+                   int64_t tiles, cudaStream_t st) {
+  using Cfg = fp8q::Ue8m0Cfg;
+  static constexpr auto kern = fp8q::gemm_fp8_ue8m0_kernel<ROW_B, OUT_BF16>;
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8Q_ERR_CUDA;
+  int units = cached[dev].load(std::memory_order_acquire);
+  if (units == 0) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(Cfg::smem_bytes)) != cudaSuccess)
+      return FP8Q_ERR_CUDA;
+    int sms = 0, per_sm = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Cfg::kThreads, Cfg::smem_bytes) !=
+            cudaSuccess || per_sm <= 0)
+      return FP8Q_ERR_CUDA;
+    units = sms * per_sm;
+    cached[dev].store(units, std::memory_order_release);
+  }
+  const int64_t grid = tiles < units ? tiles : units;
+  if (grid <= 0) return FP8Q_OK;
+  kern<<<static_cast<unsigned>(grid), Cfg::kThreads, Cfg::smem_bytes, st>>>(tmA, tmB, a);
+  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
 }  // namespace
 
 namespace fp8q {
@@ -275,6 +307,7 @@ const char* fp8q_status_string(int status) {
     case FP8Q_ERR_SHAPE: return "invalid shape or leading dimension";
     case FP8Q_ERR_ALIGN: return "pointer or leading dimension misaligned";
     case FP8Q_ERR_UNSUPPORTED: return "unsupported mode, dtype or device";
+    case FP8Q_ERR_SCALE: return "a scale is not a power of two representable as UE8M0";
     case FP8Q_ERR_CUDA: return "CUDA call failed";
     case FP8Q_ERR_TIMEOUT: return "device-side wait timed out";
     default: return "unknown status";
@@ -388,6 +421,37 @@ int fp8_gemm_blockscaled(const uint8_t* A, const float* sA, int64_t ld_sa, const
                          void* stream) {
   return fp8_gemm_blockscaled_ws(A, sA, ld_sa, B, sB, ld_sb, b_scale_mode, C, out_dtype, M, N, K,
                                  lda, ldb, ldc, nullptr, 0, stream);
+}
+
+int fp8_gemm_blockscaled_ue8m0(const uint8_t* A, const float* sA, int64_t ld_sa,
+                               const uint8_t* B, const float* sB, int64_t ld_sb, int b_scale_mode,
+                               void* C, int out_dtype, int64_t M, int64_t N, int64_t K,
+                               int64_t lda, int64_t ldb, int64_t ldc, void* stream) {
+  using Cfg = fp8q::Ue8m0Cfg;
+  if (M == 0 && N >= 0 && K >= 0) return FP8Q_OK;
+  int st = check_gemm_common(A, B, C, out_dtype, M, N, K, lda, ldb, ldc);
+  if (st != FP8Q_OK) return st;
+  if (!sA || !sB) return FP8Q_ERR_NULL;
+  if (b_scale_mode != FP8Q_BSCALE_BLOCK128x128 && b_scale_mode != FP8Q_BSCALE_ROW1x128)
+    return FP8Q_ERR_UNSUPPORTED;
+  if (ld_sa < M) return FP8Q_ERR_SHAPE;
+  if (b_scale_mode == FP8Q_BSCALE_ROW1x128 && ld_sb < N) return FP8Q_ERR_SHAPE;
+  if (!aligned(sA, 4) || !aligned(sB, 4)) return FP8Q_ERR_ALIGN;
+  CUtensorMap tmA, tmB;
+  if ((st = encode_operand(&tmA, A, K, M, lda, Cfg::kTileM)) != FP8Q_OK) return st;
+  if ((st = encode_operand(&tmB, B, K, N, ldb, Cfg::kN)) != FP8Q_OK) return st;
+  GemmArgs a{};
+  a.sA = sA; a.ld_sa = ld_sa; a.sB = sB; a.ld_sb = ld_sb; a.C = C; a.ldc = ldc;
+  a.M = M; a.N = N; a.G = static_cast<int>(K / 128); a.m_offsets = nullptr; a.num_experts = 0;
+  const int64_t tiles = ((M + Cfg::kTileM - 1) / Cfg::kTileM) * ((N + Cfg::kN - 1) / Cfg::kN);
+  if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
+  const auto s = static_cast<cudaStream_t>(stream);
+  const bool row_b = b_scale_mode == FP8Q_BSCALE_ROW1x128;
+  if (out_dtype == FP8Q_OUT_BF16)
+    return row_b ? run_gemm_ue8m0<true, true>(tmA, tmB, a, tiles, s)
+                 : run_gemm_ue8m0<false, true>(tmA, tmB, a, tiles, s);
+  return row_b ? run_gemm_ue8m0<true, false>(tmA, tmB, a, tiles, s)
+               : run_gemm_ue8m0<false, false>(tmA, tmB, a, tiles, s);
 }
 
 int fp8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, size_t* bytes) {

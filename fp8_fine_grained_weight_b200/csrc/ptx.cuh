@@ -286,4 +286,56 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Instruction descriptor, kind::mxf8f6f4 with block scaling: A = B = E4M3, both K-major,
+// dense, scale factors UE8M0.  sf_id selects the byte of the 32-bit TMEM scale cells
+// that this MMA reads (for A and for B).
+//   bits 4-5 B scale byte; 7-9 A format (0 = E4M3); 10-12 B format; 15/16 A/B major;
+//   17-22 N >> 3; 23 scale format (1 = UE8M0); 24-28 M >> 4; 29-30 A scale byte.
+__host__ __device__ constexpr uint32_t idesc_e4m3_ue8m0(int M, int N, uint32_t sf_id) {
+  return (sf_id << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (1u << 23) | (static_cast<uint32_t>(M >> 4) << 24) | (sf_id << 29);
+}
+
+// D (+)= (A x 2^(sfa - 127)) (B x 2^(sfb - 127))^T over K = 32, one CTA.  The scale
+// operands are TMEM addresses whose top two bits carry the byte selected by sf_id.
+//   A scales: row m at lane m, column sfa + m / 32.
+//   B scales: row n at column sfb + n / 32, lane n % 32 of every 32-lane sub-partition
+//   (each sub-partition reads its own copy).
+__device__ __forceinline__ void mma_f8_ue8m0(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate, uint32_t sfa,
+                                             uint32_t sfb) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// 16 consecutive TMEM columns of this warp's 32 lanes from / to registers.
+__device__ __forceinline__ void tmem_st_16cols(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
+      ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+      "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_16cols(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
 }  // namespace fp8q

@@ -45,7 +45,9 @@ typedef enum {
   FP8Q_ERR_ALIGN = 3,        /* pointer or leading dimension not 16-byte aligned as required */
   FP8Q_ERR_UNSUPPORTED = 4,  /* unknown mode / dtype, too many groups, no sm_100 device */
   FP8Q_ERR_CUDA = 5,         /* a CUDA runtime or driver call failed (launch, attribute, ...) */
-  FP8Q_ERR_TIMEOUT = 6       /* a device-side bounded wait expired (device error word only) */
+  FP8Q_ERR_TIMEOUT = 6,      /* a device-side bounded wait expired (device error word only) */
+  FP8Q_ERR_SCALE = 7         /* a scale is not a power of two in [2^-127, 2^127] where one is
+                                required (fp8_gemm_blockscaled_ue8m0; device error word only) */
 } fp8q_status;
 
 typedef enum { FP8Q_OUT_BF16 = 0, FP8Q_OUT_FP32 = 1 } fp8q_out;
@@ -113,6 +115,29 @@ int fp8_gemm_blockscaled(const uint8_t* A, const float* sA, int64_t ld_sa, const
                          const float* sB, int64_t ld_sb, int b_scale_mode, void* C, int out_dtype,
                          int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
                          void* stream);
+
+/*
+ * fp8_gemm_blockscaled for power-of-two scales, with the scaling done inside the tensor
+ * core.  why-be.co.kr wr_id=57820 para 4 and why-be.co.kr wr_id=72410 para 3 ask for
+ * tensor cores that receive the scaling factors and run the MMA with group scaling; on
+ * B200 that is the block-scaled MMA (tcgen05.mma kind::mxf8f6f4.block_scale), whose scale
+ * factors are UE8M0 bytes, i.e. powers of two.  It multiplies every 32-element K block of
+ * A and of B by its scale (exact for powers of two) and accumulates in FP32 over all of K,
+ * so no per-group promotion runs on the CUDA cores.  The quantizers' pow2 option [P2]
+ * produces such scales.
+ *
+ * Same arguments, layouts, requirements and host-side errors as fp8_gemm_blockscaled;
+ * the result is the same sum, within the same acceptance band (FP32 rounding order
+ * differs).  Every scale the call reads must be a power of two in [2^-127, 2^127]; any
+ * other value (not a power of two, zero, negative, inf, nan) is not detectable on the
+ * host: the kernel records (8 << 8) | FP8Q_ERR_SCALE in the device error word, uses 1 in
+ * its place and finishes the call (C is then not the product).  Tiles of 128 x 224; no
+ * workspace.
+ */
+int fp8_gemm_blockscaled_ue8m0(const uint8_t* A, const float* sA, int64_t ld_sa,
+                               const uint8_t* B, const float* sB, int64_t ld_sb, int b_scale_mode,
+                               void* C, int out_dtype, int64_t M, int64_t N, int64_t K,
+                               int64_t lda, int64_t ldb, int64_t ldc, void* stream);
 
 /*
  * Bytes of device workspace that fp8_gemm_blockscaled_ws can use for an M x N x K problem

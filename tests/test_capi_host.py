@@ -47,6 +47,8 @@ def test_status_strings_and_version(L):
     assert L.fp8q_status_string(0) == b"ok"
     assert b"timed out" in L.fp8q_status_string(6)
     assert L.fp8q_status_string(6 | (4 << 8)) == L.fp8q_status_string(6)
+    assert b"power of two" in L.fp8q_status_string(7)
+    assert L.fp8q_status_string(7 | (8 << 8)) == L.fp8q_status_string(7)
     assert L.fp8q_status_string(99) == b"unknown status"
 
 
@@ -75,8 +77,9 @@ def test_quant_weight_validation(L):
     assert f(P_MIS, 128, 128, 128, P16, 128, P16, 0, NULL) == 3
 
 
-def test_gemm_validation(L):
-    f = L.fp8_gemm_blockscaled
+@pytest.mark.parametrize("entry", ["fp8_gemm_blockscaled", "fp8_gemm_blockscaled_ue8m0"])
+def test_gemm_validation(L, entry):
+    f = getattr(L, entry)
     ok_args = dict(A=P16, sA=P16, ld_sa=256, B=P16, sB=P16, ld_sb=0, mode=0, C=P16, out=0,
                    M=256, N=256, K=256, lda=256, ldb=256, ldc=256)
 

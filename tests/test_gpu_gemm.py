@@ -27,8 +27,9 @@ def fq():
 
 
 def _dense_case(fq, a_bits, b_bits, pow2_a, pow2_b, out_fp32, b_rowwise=False, rows=None,
-                name="dense"):
-    """Quantize on both sides, check the codes, run the GEMM, compare (sampled) rows."""
+                name="dense", ue8m0=False):
+    """Quantize on both sides, check the codes, run the GEMM, compare (sampled) rows.
+    ue8m0: the power-of-two-scale GEMM that scales inside the tensor core."""
     import torch
     a, b = to_dev_bf16(a_bits), to_dev_bf16(b_bits)
     qa, sa = fq.quant_act_1x128(a, pow2_a)
@@ -37,7 +38,8 @@ def _dense_case(fq, a_bits, b_bits, pow2_a, pow2_b, out_fp32, b_rowwise=False, r
     else:
         qb, sb = fq.quant_weight_128x128(b, pow2_b)
     out_dtype = torch.float32 if out_fp32 else torch.bfloat16
-    C = fq.gemm_blockscaled(qa, sa, qb, sb, out_dtype=out_dtype, b_rowwise=b_rowwise)
+    gemm = fq.gemm_blockscaled_ue8m0 if ue8m0 else fq.gemm_blockscaled
+    C = gemm(qa, sa, qb, sb, out_dtype=out_dtype, b_rowwise=b_rowwise)
     torch.cuda.synchronize()
     assert fq.device_error() == 0
 
@@ -282,3 +284,99 @@ def test_nopromo_matches_oracle_on_rowwise_codes(fq):
     # no acceptance band is claimed for this variant; it must still be a close FP32 result
     mx, _ = rel_err_stats(host(C), C_ref, T)
     assert mx < 1e-3
+
+
+# ------------------------------------------------------- power-of-two scales in the MMA
+
+def _spread_scales(rng, bits, rows_per_block, span=24):
+    """Multiply each (row block, 128-column group) of a bf16 matrix by 2^u, u uniform in
+    [-span, span], so that neighbouring rows / columns / groups get very different
+    power-of-two scales (a wrong row, column or group in the scale layout shows up as an
+    error of a power of two)."""
+    R, K = bits.shape
+    x = workloads.bf16_bits_to_fp32(bits).astype(np.float64)
+    nb, G = -(-R // rows_per_block), K // 128
+    u = rng.integers(-span, span + 1, size=(nb, G))
+    f = np.repeat(np.repeat(np.exp2(u), rows_per_block, axis=0)[:R], 128, axis=1)
+    return workloads.fp32_to_bf16_bits((x * f).astype(np.float32))
+
+
+def test_ue8m0_tiny_fp32(fq):
+    w = workloads.tiny()
+    C, C_ref, T, _ = _dense_case(fq, w.gen_a(), w.gen_b(), True, True, True, name="ue8m0 tiny",
+                                 ue8m0=True)
+    mx, _ = rel_err_stats(C, C_ref, T)
+    assert mx <= 2e-5
+
+
+def test_ue8m0_unit_scale_integers_exact(fq):
+    """Small E4M3 integers with unit scales (UE8M0 byte 127): the exact integer product."""
+    import torch
+    rng = workloads.rng_for(1, 9)
+    qa, ia = workloads.small_int_e4m3_codes(rng, (128, 512))
+    qb, ib = workloads.small_int_e4m3_codes(rng, (384, 512))   # 224 + a ragged 160
+    sa = np.ones((4, 128), np.float32)
+    sb = np.ones((3, 4), np.float32)
+    C = fq.gemm_blockscaled_ue8m0(to_dev(qa), to_dev(sa), to_dev(qb), to_dev(sb),
+                                  out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert fq.device_error() == 0
+    assert_bytes_equal("ue8m0 unit-scale C", host(C), (ia @ ib.T).astype(np.float32))
+
+
+@pytest.mark.parametrize("out_fp32", [True, False])
+@pytest.mark.parametrize("M,N,K", [(300, 512, 640), (129, 1280, 384)])
+def test_ue8m0_spread_scales(fq, M, N, K, out_fp32):
+    """Per-row-tile / per-block scales spread over 2^-24 .. 2^24, group counts that are not
+    multiples of 4 (K = 640, 384: a scale slot holds four groups), ragged M and N."""
+    rng = np.random.default_rng(M * 7 + N + K)
+    a = _spread_scales(rng, workloads.normal_bf16(rng, (M, K), 1.0, 0.001), 1)
+    b = _spread_scales(rng, workloads.normal_bf16(rng, (N, K), 0.02), 128)
+    _dense_case(fq, a, b, True, True, out_fp32, name=f"ue8m0 spread {M}x{N}x{K}", ue8m0=True)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 128, 128), (129, 256, 128), (200, 384, 640),
+                                   (257, 512, 256), (64, 128, 1024), (300, 1280, 384),
+                                   (513, 2048, 1152)])
+def test_ue8m0_ragged_shapes(fq, M, N, K):
+    rng = np.random.default_rng(M + 3 * N + 7 * K)
+    a = workloads.normal_bf16(rng, (M, K), 1.0, 0.01)
+    b = workloads.normal_bf16(rng, (N, K), 0.02)
+    _dense_case(fq, a, b, True, True, False, name=f"ue8m0 ragged {M}x{N}x{K}", ue8m0=True)
+
+
+@pytest.mark.parametrize("M,N,K", [(77, 256, 512), (128, 384, 384)])
+def test_ue8m0_rowwise_b_scales(fq, M, N, K):
+    rng = np.random.default_rng(M * N + 1)
+    a = _spread_scales(rng, workloads.normal_bf16(rng, (M, K), 1e-3), 1, span=8)
+    b = _spread_scales(rng, workloads.normal_bf16(rng, (N, K), 1.0), 1, span=8)
+    _dense_case(fq, a, b, True, True, True, b_rowwise=True, name="ue8m0 row-b", ue8m0=True)
+
+
+def test_ue8m0_dense_full_size_sampled_rows(fq):
+    """The dense workload (power-of-two scales) at full size through the tensor-core-scaled
+    GEMM; 96 sampled rows spanning every M tile and the last row."""
+    w = workloads.dense()
+    rng = np.random.default_rng(10)
+    rows = np.unique(np.concatenate([rng.choice(w.M, 94, replace=False), [0, w.M - 1]]))
+    _dense_case(fq, w.gen_a(), w.gen_b(), True, True, False, rows=rows, name="ue8m0 dense full",
+                ue8m0=True)
+
+
+def test_ue8m0_rejects_scales_that_are_not_powers_of_two(fq):
+    """FP32 (non power-of-two) scales cannot be UE8M0 bytes: the kernel finishes, records
+    (8 << 8) | FP8Q_ERR_SCALE in the device error word, and the next call is clean."""
+    import torch
+    w = workloads.tiny()
+    qa, sa = fq.quant_act_1x128(to_dev_bf16(w.gen_a()), False)
+    qb, sb = fq.quant_weight_128x128(to_dev_bf16(w.gen_b()), False)
+    assert not bool(torch.all(torch.frexp(sa)[0] == 0.5))     # some scale is not 2^e
+    fq.gemm_blockscaled_ue8m0(qa, sa, qb, sb, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert fq.device_error() == (8 << 8) | 7
+    assert fq.device_error() == 0                                # read and cleared
+    qa2, sa2 = fq.quant_act_1x128(to_dev_bf16(w.gen_a()), True)
+    qb2, sb2 = fq.quant_weight_128x128(to_dev_bf16(w.gen_b()), True)
+    fq.gemm_blockscaled_ue8m0(qa2, sa2, qb2, sb2, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert fq.device_error() == 0
