@@ -157,6 +157,13 @@ def run_gpu(args, rank, world):
     flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
+    # The GEMM of the step: with power-of-two scales on both operands the tensor core
+    # applies them (fp8_gemm_blockscaled_ue8m0); otherwise the per-group promoted GEMM.
+    path = gemm_path(args, w)
+    gemms = {"ue8m0": lambda: fq.gemm_blockscaled_ue8m0(qA, sA, qW, sW, out=C),
+             "promoted": lambda: fq.gemm_blockscaled(qA, sA, qW, sW, out=C)}
+    gemm = gemms[path]
+
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
@@ -166,7 +173,7 @@ def run_gpu(args, rank, world):
         fq.quant_weight_128x128(W, w.pow2_b, out=(qW, sW))
         if ev is not None:
             ev[2].record(stream)
-        fq.gemm_blockscaled(qA, sA, qW, sW, out=C)
+        gemm()
         if ev is not None:
             ev[3].record(stream)
 
@@ -212,15 +219,27 @@ def run_gpu(args, rank, world):
     w_bytes = N * K * 2 + N * K + (N // 128) * G * 4
     value = world * flops / (ms_step * 1e-3) / 1e12
 
+    kernel = GEMM_KERNEL[path]
     traffic = None
-    tp = os.path.join(ROOT, "profiles", "gemm_dense_traffic.json")
+    tp = os.path.join(ROOT, "profiles", f"{kernel}_dense_traffic.json")
     if os.path.exists(tp):
         try:
             tj = json.load(open(tp))
-            if tj.get("workload") == w.name and tj.get("kernel_rev") == kernel_rev():
+            if (tj.get("workload") == w.name and tj.get("kernel") == kernel
+                    and tj.get("kernel_rev") == kernel_rev()):
                 traffic = tj.get("dram_bytes_per_launch")
         except Exception:
             traffic = None
+    # both GEMM paths on this step's operands (L2 flushed before each launch)
+    paths = {}
+    for name in (("ue8m0", "promoted") if w.pow2_a and w.pow2_b else ("promoted",)):
+        t = _time_ms(gemms[name], 20, flush_l2)
+        tf = flops / (t * 1e-3) / 1e12
+        paths[name] = {"kernel": GEMM_KERNEL[name], "ms": round(t, 5), "tflops": round(tf, 1),
+                       "frac_of_fp8_peak": round(tf / fp8_peak, 4)}
+    if fq.device_error():
+        raise RuntimeError("device error word set after the GEMM path timings")
+    gemm_launches = 1 if path == "ue8m0" else (2 if fq.workspace_bytes(M, N, K) else 1)
 
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
@@ -232,7 +251,9 @@ def run_gpu(args, rank, world):
                    "parallelism": f"replicas x{world} (dense: each GPU its own 4096-token batch)",
                    "l2": "flush between steps (512 MB write, then read back), outside the per-step events"},
         "kernels_ms": {"quant_act_1x128": round(ms_act, 5), "quant_weight_128x128": round(ms_w, 5),
-                       "gemm_blockscaled": round(ms_gemm, 5)},
+                       kernel: round(ms_gemm, 5)},
+        "gemm_path": path,
+        "gemm_paths": paths,
         "gemm_tflops": round(gemm_tflops, 1),
         "gemm_frac_of_fp8_peak": round(gemm_tflops / fp8_peak, 4),
         "gemm_frac_of_fp8_spec_4500": round(gemm_tflops / 4500.0, 4),
@@ -243,9 +264,9 @@ def run_gpu(args, rank, world):
         "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 1),
                      "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
                      "frac": round(gemm_tflops / fp8_peak, 4), "traffic": traffic,
-                     "kernel": "gemm_blockscaled",
+                     "kernel": kernel,
                      "peak_source": f"{peak_src} bf16 burst {bf16_burst} x {FP8_PER_BF16} (fp8:bf16)"},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": (2 + gemm_launches) * args.steps,
         "clocks": clk.summary(),
     }
 
@@ -435,7 +456,7 @@ def accumulation_study(fq, rows_sampled=32):
             "results": res}
 
 
-def profile_case(name: str, launches: int = 3):
+def profile_case(args, name: str, launches: int = 3):
     """A few launches of one workload's kernels on device-drawn inputs (for ncu captures)."""
     import torch
     import fp8_fine_grained_weight_b200 as fq
@@ -454,7 +475,10 @@ def profile_case(name: str, launches: int = 3):
         qA, sA = fq.quant_act_1x128(A, w.pow2_a)
         qB, sB = fq.quant_act_1x128(B, w.pow2_b) if w.b_rowwise else fq.quant_weight_128x128(B, w.pow2_b)
         C = torch.empty((w.M, w.N), dtype=torch.float32 if w.out_fp32 else torch.bfloat16, device="cuda")
-        run = lambda: fq.gemm_blockscaled(qA, sA, qB, sB, b_rowwise=w.b_rowwise, out=C)
+        if gemm_path(args, w) == "ue8m0":
+            run = lambda: fq.gemm_blockscaled_ue8m0(qA, sA, qB, sB, b_rowwise=w.b_rowwise, out=C)
+        else:
+            run = lambda: fq.gemm_blockscaled(qA, sA, qB, sB, b_rowwise=w.b_rowwise, out=C)
     for _ in range(launches):
         run()
     torch.cuda.synchronize()
@@ -463,11 +487,24 @@ def profile_case(name: str, launches: int = 3):
     print(json.dumps({"profile_case": w.name, "launches": launches}), flush=True)
 
 
+GEMM_KERNEL = {"ue8m0": "gemm_blockscaled_ue8m0", "promoted": "gemm_blockscaled"}
+
+
+def gemm_path(args, w) -> str:
+    """The dense step's GEMM: the tensor-core-scaled one when both operands have
+    power-of-two scales (unless --gemm says otherwise), else the promoted one."""
+    if args.gemm != "auto":
+        if args.gemm == "ue8m0" and not (w.pow2_a and w.pow2_b):
+            raise SystemExit("--gemm ue8m0 needs power-of-two scales on both operands")
+        return args.gemm
+    return "ue8m0" if (w.pow2_a and w.pow2_b) else "promoted"
+
+
 def kernel_rev() -> str:
     """Short hash of the kernel sources, to tie stored ncu counters to the code they measured."""
     import hashlib
     h = hashlib.sha1()
-    for f in ("ptx.cuh", "quant.cuh", "gemm.cuh", "fp8q.cu"):
+    for f in ("ptx.cuh", "quant.cuh", "gemm.cuh", "gemm_ue8m0.cuh", "fp8q.cu"):
         h.update(open(os.path.join(ROOT, "fp8_fine_grained_weight_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:12]
 
@@ -556,6 +593,9 @@ def main():
                     help="the dense workload timed as one step (the bench line)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--gemm", default="auto", choices=["auto", "ue8m0", "promoted"],
+                    help="dense GEMM: auto = tensor-core scaling when both operands have "
+                         "power-of-two scales, else per-group promotion")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-check", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' timings")
@@ -567,7 +607,7 @@ def main():
     if args.profile_case:
         import torch
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-        profile_case(args.profile_case)
+        profile_case(args, args.profile_case)
         return
 
     if args.impl == "reference":
