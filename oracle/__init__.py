@@ -53,6 +53,8 @@ def lib() -> ctypes.CDLL:
         L.orc_quant_rowwise.argtypes = [vp, i64, i64, i64, vp, i64, vp, i32]
         L.orc_quant_rowwise.restype = None
         L.orc_gemm_triple.argtypes = [vp, vp, i64, vp, vp, i64, i32, i64, i64, i64, vp, vp]
+        L.orc_quant_tensorwise.restype = None
+        L.orc_quant_tensorwise.argtypes = [vp, i64, i64, i64, vp, i64, vp, i32]
         L.orc_gemm_triple.restype = None
         _lib = L
     return _lib
@@ -124,6 +126,17 @@ def quant_rowwise(x_bits: np.ndarray, pow2: bool = False):
     s = np.empty((M,), dtype=np.float32)
     lib().orc_quant_rowwise(_ptr(x), M, K, K, _ptr(q), K, _ptr(s), int(bool(pow2)))
     return q, s
+
+
+def quant_tensorwise(x_bits: np.ndarray, pow2: bool = False):
+    """One scale for the whole tensor (the coarse baseline of the outlier study).
+    Returns (q uint8 [R, C], s float)."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    R, C = x.shape
+    q = np.empty((R, C), dtype=np.uint8)
+    s = np.zeros((1,), dtype=np.float32)
+    lib().orc_quant_tensorwise(_ptr(x), R, C, C, _ptr(q), C, _ptr(s), int(bool(pow2)))
+    return q, float(s[0])
 
 
 # ----------------------------------------------------------------------------------

@@ -197,6 +197,31 @@ void orc_quant_rowwise(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
 }
 
 /* ---------------------------------------------------------------------- */
+/* one scale for the whole tensor (the coarse baseline)                    */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * The per-tensor scaling that fine-grained quantization replaces.  the-good.kr
+ * wr_id=2169793 para 4: the usual practice maps the maximum absolute value of the
+ * whole input tensor to the largest FP8 value, which leaves low-precision training
+ * very sensitive to activation outliers; pkd.ac.th webboard 78017 para 1 answers
+ * with scaling at a finer grain.  Same scale rule as the tiles, with the amax over
+ * all R x C elements; *s receives the single scale.
+ */
+void orc_quant_tensorwise(const uint16_t* x, int64_t R, int64_t C, int64_t ldx,
+                          uint8_t* q, int64_t ldq, float* s, int pow2) {
+    float amax = 0.0f, sc;
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t c = 0; c < C; ++c) amax = amax_update(amax, bf16_to_f32(x[r * ldx + c]));
+    sc = orc_scale_from_amax(amax, pow2);
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t c = 0; c < C; ++c)
+            q[r * ldq + c] = orc_e4m3_encode(bf16_to_f32(x[r * ldx + c]) / sc);
+    *s = sc;
+}
+
+/* ---------------------------------------------------------------------- */
 /* brute-force GEMM (tiny shapes)                                          */
 /* ---------------------------------------------------------------------- */
 
