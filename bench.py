@@ -401,6 +401,35 @@ def config_throughput(fq, flush_l2, reps=10):
     out["wgrad"] = {"workload": w.name, "gemm_ms": round(t_g, 4), "gemm_tflops": round(tf, 1),
                     "gemm_frac_of_fp8_peak": round(tf / fp8_peak, 4),
                     "quant_act_gbs": round(w.M * w.K * (3 + 4 / 128) / (t_a * 1e-3) / 1e9, 1)}
+    del A, B, qA, sA, qB, sB, C
+    # rows and the transposed copy in one pass: a gradient dY of 16384 tokens x 7168
+    T, Nc = 16384, 7168
+    dY = _dev_normal((T, Nc), 1e-3, 6001)
+    bufs = fq.quant_act_dual(dY, False)
+    t_d = _time_ms(lambda: fq.quant_act_dual(dY, False, out=bufs), reps, flush_l2)
+    dual_bytes = T * Nc * (2 + 2 + 8 / 128)
+    out["quant_dual"] = {"workload": f"quant_act_dual_{T}x{Nc}", "ms": round(t_d, 4),
+                         "gbs": round(dual_bytes / (t_d * 1e-3) / 1e9, 1),
+                         "frac_of_hbm": round(dual_bytes / (t_d * 1e-3) / 1e9 / hbm, 4),
+                         "algorithmic_bytes": int(dual_bytes)}
+    del dY, bufs
+    # FP8 linear layer, one forward + backward (Fprop, Dgrad, Wgrad), dense shapes, pow2
+    from fp8_fine_grained_weight_b200.linear import fp8_linear
+    Tl, Kl, Nl = 4096, 7168, 7168
+    x = _dev_normal((Tl, Kl), 1.0, 6002).requires_grad_(True)
+    wl = _dev_normal((Nl, Kl), 0.006, 6003).requires_grad_(True)
+    dyl = _dev_normal((Tl, Nl), 1e-3, 6004)
+
+    def fwd_bwd():
+        x.grad = None
+        wl.grad = None
+        fp8_linear(x, wl, True).backward(dyl)
+
+    t_l = _time_ms(fwd_bwd, reps, flush_l2)
+    tf = 3 * 2 * Tl * Kl * Nl / (t_l * 1e-3) / 1e12
+    out["fp8_linear"] = {"workload": f"fp8_linear_fwd_bwd_{Tl}x{Kl}x{Nl}_pow2", "ms": round(t_l, 4),
+                         "tflops_3_gemms": round(tf, 1), "frac_of_fp8_peak": round(tf / fp8_peak, 4),
+                         "launches": 7}
     return out
 
 

@@ -35,6 +35,9 @@ SIGNATURES = {
     "fp8q_quant_act_1x128": (_i32, [_vp, _i64, _i64, _i64, _vp, _i64, _vp, _i64, _i32, _vp]),
     "fp8q_quant_weight_128x128": (_i32, [_vp, _i64, _i64, _i64, _vp, _i64, _vp, _i32, _vp]),
     "fp8q_quant_rowwise": (_i32, [_vp, _i64, _i64, _i64, _vp, _i64, _vp, _i32, _vp]),
+    "fp8q_transpose_blocks": (_i32, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _i64, _vp]),
+    "fp8q_quant_act_dual": (_i32, [_vp, _i64, _i64, _i64, _vp, _i64, _vp, _i64, _vp, _i64,
+                                   _vp, _i64, _i32, _vp]),
     "fp8_gemm_blockscaled": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _i32, _vp, _i32,
                                     _i64, _i64, _i64, _i64, _i64, _i64, _vp]),
     "fp8_gemm_blockscaled_ue8m0": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _i32, _vp, _i32,
@@ -121,6 +124,44 @@ def quant_act_1x128(x: torch.Tensor, pow2: bool = False, ld_scale: Optional[int]
     _call("fp8q_quant_act_1x128", x.data_ptr(), M, K, x.stride(0), q.data_ptr(), q.stride(0),
           s.data_ptr(), ld, int(bool(pow2)), _stream(x))
     return q, s
+
+
+def quant_act_dual(x: torch.Tensor, pow2: bool = False, out=None):
+    """Rows and columns from one read: x bf16 [M, K] (M, K multiples of 128) ->
+    (q uint8 [M, K], s fp32 [K/128, M], qt uint8 [K, M], st fp32 [M/128, K]), where (q, s)
+    is quant_act_1x128(x) and (qt, st) is quant_act_1x128 of x transposed."""
+    _need(x, torch.bfloat16, "x", 2)
+    M, K = x.shape
+    if out is None:
+        q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+        s = torch.empty((K // 128, M), dtype=torch.float32, device=x.device)
+        qt = torch.empty((K, M), dtype=torch.uint8, device=x.device)
+        st = torch.empty((M // 128, K), dtype=torch.float32, device=x.device)
+    else:
+        q, s, qt, st = out
+    _call("fp8q_quant_act_dual", x.data_ptr(), M, K, x.stride(0), q.data_ptr(), q.stride(0),
+          s.data_ptr(), s.stride(0), qt.data_ptr(), qt.stride(0), st.data_ptr(), st.stride(0),
+          int(bool(pow2)), _stream(x))
+    return q, s, qt, st
+
+
+def transpose_blocks(q: torch.Tensor, s: torch.Tensor, out=None):
+    """q uint8 [N, K], s fp32 [N/128, K/128] (128x128 blocks) -> (q^T [K, N], s^T [K/128, N/128]):
+    the 128x128 quantization of the transposed matrix."""
+    q = _u8(q)
+    _need(q, torch.uint8, "q", 2)
+    _need(s, torch.float32, "s", 2)
+    N, K = q.shape
+    if not s.is_contiguous():
+        raise ValueError("s must be contiguous")
+    if out is None:
+        qt = torch.empty((K, N), dtype=torch.uint8, device=q.device)
+        st = torch.empty((K // 128, N // 128), dtype=torch.float32, device=q.device)
+    else:
+        qt, st = out
+    _call("fp8q_transpose_blocks", q.data_ptr(), s.data_ptr(), N, K, q.stride(0), qt.data_ptr(),
+          st.data_ptr(), qt.stride(0), _stream(q))
+    return qt, st
 
 
 def quant_weight_128x128(w: torch.Tensor, pow2: bool = False,

@@ -347,6 +347,57 @@ int fp8q_quant_act_1x128(const void* x, int64_t M, int64_t K, int64_t ldx, uint8
   return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
+int fp8q_quant_act_dual(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
+                        int64_t ldq, float* s, int64_t ld_s, uint8_t* qt, int64_t ldqt,
+                        float* st, int64_t ld_st, int pow2_scale, void* stream) {
+  if (M < 0 || K < 0) return FP8Q_ERR_SHAPE;
+  if (M == 0 || K == 0) return FP8Q_OK;
+  if (!x || !q || !s || !qt || !st) return FP8Q_ERR_NULL;
+  if (M % 128 != 0 || K % 128 != 0 || ldx < K || ldq < K || ld_s < M || ldqt < M || ld_st < K)
+    return FP8Q_ERR_SHAPE;
+  if (ldx % 8 != 0 || ldq % 8 != 0 || ldqt % 16 != 0 || !aligned(x, 16) || !aligned(q, 8) ||
+      !aligned(qt, 16) || !aligned(s, 4) || !aligned(st, 4))
+    return FP8Q_ERR_ALIGN;
+  if (K / 128 > 65535 || M / 128 > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
+  static std::atomic<unsigned long long> ready{0};   // per-device bit: attributes set
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8Q_ERR_CUDA;
+  if (!(ready.load(std::memory_order_acquire) & (1ull << dev))) {
+    if (cudaFuncSetAttribute(fp8q::quant_act_dual_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fp8q::kDualSmem) != cudaSuccess ||
+        cudaFuncSetAttribute(fp8q::quant_act_dual_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fp8q::kDualSmem) != cudaSuccess)
+      return FP8Q_ERR_CUDA;
+    ready.fetch_or(1ull << dev, std::memory_order_acq_rel);
+  }
+  dim3 grid(static_cast<unsigned>(M / 128), static_cast<unsigned>(K / 128));
+  auto stm = static_cast<cudaStream_t>(stream);
+  const auto* xs = static_cast<const uint16_t*>(x);
+  if (pow2_scale)
+    fp8q::quant_act_dual_kernel<true><<<grid, 256, fp8q::kDualSmem, stm>>>(xs, ldx, q, ldq, s, ld_s, qt,
+                                                                           ldqt, st, ld_st);
+  else
+    fp8q::quant_act_dual_kernel<false><<<grid, 256, fp8q::kDualSmem, stm>>>(xs, ldx, q, ldq, s, ld_s, qt,
+                                                                            ldqt, st, ld_st);
+  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+int fp8q_transpose_blocks(const uint8_t* q, const float* s, int64_t N, int64_t K, int64_t ldq,
+                          uint8_t* qt, float* st, int64_t ldqt, void* stream) {
+  if (N < 0 || K < 0) return FP8Q_ERR_SHAPE;
+  if (N == 0 || K == 0) return FP8Q_OK;
+  if (!q || !s || !qt || !st) return FP8Q_ERR_NULL;
+  if (N % 128 != 0 || K % 128 != 0 || ldq < K || ldqt < N) return FP8Q_ERR_SHAPE;
+  if (ldq % 16 != 0 || ldqt % 16 != 0 || !aligned(q, 16) || !aligned(qt, 16) || !aligned(s, 4) ||
+      !aligned(st, 4))
+    return FP8Q_ERR_ALIGN;
+  if (N / 128 > 65535 || K / 128 > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
+  dim3 grid(static_cast<unsigned>(K / 128), static_cast<unsigned>(N / 128));
+  fp8q::transpose_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      q, s, ldq, static_cast<int>(K / 128), qt, st, ldqt, static_cast<int>(N / 128));
+  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
 int fp8q_quant_weight_128x128(const void* w, int64_t N, int64_t K, int64_t ldw, uint8_t* q,
                               int64_t ldq, float* scales, int pow2_scale, void* stream) {
   if (N < 0 || K < 0) return FP8Q_ERR_SHAPE;

@@ -202,6 +202,188 @@ __global__ void __launch_bounds__(256) quant_act_1x128_kernel(const uint16_t* __
   }
 }
 
+// ---------------------------------------------------------------- rows and columns in one pass
+//
+// One HBM read of a bf16 activation X [M, K] produces both
+//   q  / s : the 1x128 quantization of X (along K; for Fprop and Dgrad), and
+//   qt / st: the 1x128 quantization of X^T (along M, i.e. 128x1 tiles of X; for Wgrad),
+// qt [K, M] with row stride ldqt, st group-major [M/128][ldst].  why-be.co.kr wr_id=57820
+// para 4 and why-be.co.kr wr_id=72410 para 3 note that the quantization pass reads the
+// activations from HBM and that the transposed copy needed by the backward pass costs
+// another round trip; this kernel reads each element once for both.
+//
+// Grid (M/128, K/128), 256 threads, one 128x128 tile of X per block:
+//  rows:    as quant_act_1x128_kernel (teams of 4 lanes per row, 16 rows per warp), all
+//           eight 16-byte loads of a thread issued before any arithmetic; the tile is
+//           kept in shared memory (row pitch 256 bytes);
+//  columns: thread t owns the column pair 2 (t % 64), +1 and rows 32 (t / 64) .. + 31 of
+//           the tile (32-bit shared loads); the four quarters' amax meet in shared memory;
+//           the codes are staged transposed in the tile's space once every thread has
+//           read it (row pitch kDualPitch bytes) and written as 128-byte column segments.
+constexpr int kDualPitch = 144;                     // 128 codes + 16
+constexpr int kDualSmem = 128 * 256 + 4 * 64 * 4;  // tile (reused for the codes) + amax parts
+static_assert(128 * kDualPitch <= 128 * 256, "codes fit in the tile's space");
+
+template <bool POW2>
+__global__ void __launch_bounds__(256, 5) quant_act_dual_kernel(const uint16_t* __restrict__ x,
+                                                             int64_t ldx, uint8_t* __restrict__ q,
+                                                             int64_t ldq, float* __restrict__ s,
+                                                             int64_t lds, uint8_t* __restrict__ qt,
+                                                             int64_t ldqt, float* __restrict__ st,
+                                                             int64_t ldst) {
+  extern __shared__ __align__(16) uint8_t dual_smem[];
+  uint8_t* tile = dual_smem;                               // bf16 [128][128], then E4M3 codes
+  uint32_t* part = reinterpret_cast<uint32_t*>(dual_smem + 128 * 256);   // [4][64] amax pairs
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int l4 = lane & 3;
+  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * 128;
+  const int64_t k0 = static_cast<int64_t>(blockIdx.y) * 128;
+  const int64_t g = blockIdx.y;
+
+  // ---- rows: both passes' loads first
+  uint4 v[2][4];
+#pragma unroll
+  for (int pass = 0; pass < 2; ++pass) {
+    const int64_t m = m0 + warp * 16 + pass * 8 + (lane >> 2);
+    const uint16_t* src = x + m * ldx + k0 + l4 * 8;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[pass][j] = ldg_stream(src + 32 * j);
+  }
+#pragma unroll
+  for (int pass = 0; pass < 2; ++pass) {
+    const int r = warp * 16 + pass * 8 + (lane >> 2);      // row inside the tile
+    const int64_t m = m0 + r;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(tile + r * 256 + (l4 + 4 * j) * 16) = v[pass][j];
+    float a = amax_vectors(v[pass]);
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+    const float sc = tile_scale(a, POW2);
+    const Quotient qd(sc);
+    uint2 o[4];
+    quant_vectors(v[pass], qd, o);
+    uint8_t* dst = q + m * ldq + k0 + l4 * 8;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) stg_u2(dst + 32 * j, o[j]);
+    if (l4 == 0) s[g * lds + m] = sc;
+  }
+  __syncthreads();
+
+  // ---- columns 2p, 2p+1 over rows 32h .. 32h + 31
+  const int p = threadIdx.x & 63, h = threadIdx.x >> 6;
+  const uint32_t* words = reinterpret_cast<const uint32_t*>(tile) + p;   // row r: words[64 r]
+  uint32_t mx = 0;
+#pragma unroll 8
+  for (int r = 0; r < 32; ++r) mx = __vmaxu2(mx, words[(32 * h + r) * 64] & 0x7FFF7FFFu);
+  part[h * 64 + p] = mx;
+  __syncthreads();
+  const uint32_t mall = __vmaxu2(__vmaxu2(part[p], part[64 + p]), __vmaxu2(part[128 + p], part[192 + p]));
+  const float sc_lo = tile_scale(__uint_as_float((mall & 0xFFFFu) << 16), POW2);
+  const float sc_hi = tile_scale(__uint_as_float(mall & 0xFFFF0000u), POW2);
+  const Quotient q_lo(sc_lo), q_hi(sc_hi);
+  uint32_t c_lo[8], c_hi[8];                               // 32 codes of each column
+  // the quotient rule is picked once for the pair (both columns share it but for rare
+  // scales that happen to be powers of two, or tiny ones)
+  auto codes_with = [&](auto f_lo, auto f_hi) {
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      const int r = 32 * h + 4 * w;
+      const uint32_t w0 = words[r * 64], w1 = words[(r + 1) * 64];
+      const uint32_t w2 = words[(r + 2) * 64], w3 = words[(r + 3) * 64];
+      c_lo[w] = cvt_e4m3x2(f_lo(bf16lo(w0)), f_lo(bf16lo(w1))) |
+                (cvt_e4m3x2(f_lo(bf16lo(w2)), f_lo(bf16lo(w3))) << 16);
+      c_hi[w] = cvt_e4m3x2(f_hi(bf16hi(w0)), f_hi(bf16hi(w1))) |
+                (cvt_e4m3x2(f_hi(bf16hi(w2)), f_hi(bf16hi(w3))) << 16);
+    }
+  };
+  if (q_lo.mode == kCorrected && q_hi.mode == kCorrected) {
+    const float r_lo = q_lo.r, s_lo = q_lo.s, r_hi = q_hi.r, s_hi = q_hi.s;
+    codes_with(
+        [r_lo, s_lo](float xv) {
+          const float q0 = __fmul_rn(xv, r_lo);
+          return copysignf(__fmaf_rn(__fmaf_rn(-q0, s_lo, xv), r_lo, q0), xv);
+        },
+        [r_hi, s_hi](float xv) {
+          const float q0 = __fmul_rn(xv, r_hi);
+          return copysignf(__fmaf_rn(__fmaf_rn(-q0, s_hi, xv), r_hi, q0), xv);
+        });
+  } else if (q_lo.mode == kExactRcp && q_hi.mode == kExactRcp) {
+    const float r_lo = q_lo.r, r_hi = q_hi.r;
+    codes_with([r_lo](float xv) { return __fmul_rn(xv, r_lo); },
+               [r_hi](float xv) { return __fmul_rn(xv, r_hi); });
+  } else {
+    codes_with([&q_lo](float xv) { return q_lo(xv); }, [&q_hi](float xv) { return q_hi(xv); });
+  }
+  if (h == 0) {
+    float* sdst = st + (m0 / 128) * ldst + k0 + 2 * p;
+    sdst[0] = sc_lo;
+    sdst[1] = sc_hi;
+  }
+  __syncthreads();                                         // every thread is done reading the tile
+  uint8_t* codes = tile;                                   // [128 columns][kDualPitch]
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    *reinterpret_cast<uint4*>(codes + (2 * p) * kDualPitch + 32 * h + 16 * j) =
+        make_uint4(c_lo[4 * j], c_lo[4 * j + 1], c_lo[4 * j + 2], c_lo[4 * j + 3]);
+    *reinterpret_cast<uint4*>(codes + (2 * p + 1) * kDualPitch + 32 * h + 16 * j) =
+        make_uint4(c_hi[4 * j], c_hi[4 * j + 1], c_hi[4 * j + 2], c_hi[4 * j + 3]);
+  }
+  __syncthreads();
+  // 128 columns x 128 codes: each group of 8 threads writes one 128-byte column segment
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int idx = j * 256 + threadIdx.x;
+    const int cc = idx >> 3, chunk = idx & 7;
+    const uint4 val = *reinterpret_cast<const uint4*>(codes + cc * kDualPitch + chunk * 16);
+    *reinterpret_cast<uint4*>(qt + (k0 + cc) * ldqt + m0 + chunk * 16) = val;
+  }
+}
+
+// ---------------------------------------------------------------- transposed weight blocks
+//
+// qt = q^T and st = s^T for a matrix quantized in 128x128 blocks.  Block quantization is
+// symmetric under transposition (a block's amax is that of its transpose), so these are
+// exactly the codes and scales of the transposed bf16 matrix: the operand a Dgrad GEMM
+// (dX = dY W) needs, without requantizing from bf16.  Grid (K/128, N/128), 256 threads,
+// one block per CTA through shared memory (row pitch 132 bytes).
+constexpr int kTrPitch = 132;
+
+__global__ void __launch_bounds__(256) transpose_blocks_kernel(const uint8_t* __restrict__ q,
+                                                               const float* __restrict__ s,
+                                                               int64_t ldq, int G,
+                                                               uint8_t* __restrict__ qt,
+                                                               float* __restrict__ st,
+                                                               int64_t ldqt, int NB) {
+  __shared__ __align__(16) uint8_t blk[128 * kTrPitch];
+  const int64_t g = blockIdx.x, nb = blockIdx.y;
+  const uint8_t* src = q + nb * 128 * ldq + g * 128;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {                     // 128 rows x 128 B, 16 B per thread
+    const int idx = j * 256 + threadIdx.x;
+    const int r = idx >> 3, chunk = idx & 7;
+    const uint4 v = *reinterpret_cast<const uint4*>(src + r * ldq + chunk * 16);
+    uint32_t* d = reinterpret_cast<uint32_t*>(blk + r * kTrPitch + chunk * 16);
+    d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
+  }
+  __syncthreads();
+  uint8_t* dst = qt + g * 128 * ldqt + nb * 128;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {                     // output row c = input column c
+    const int idx = j * 256 + threadIdx.x;
+    const int c = idx >> 3, chunk = idx & 7;
+    uint32_t w[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int r = chunk * 16 + 4 * b;
+      w[b] = static_cast<uint32_t>(blk[r * kTrPitch + c]) | (static_cast<uint32_t>(blk[(r + 1) * kTrPitch + c]) << 8) |
+             (static_cast<uint32_t>(blk[(r + 2) * kTrPitch + c]) << 16) |
+             (static_cast<uint32_t>(blk[(r + 3) * kTrPitch + c]) << 24);
+    }
+    *reinterpret_cast<uint4*>(dst + c * ldqt + chunk * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  if (threadIdx.x == 0) st[g * NB + nb] = s[nb * G + g];
+}
+
 // ---------------------------------------------------------------- 128x128 weight blocks
 //
 // Grid (G, N/128): one 256-thread block per 128x128 block.  Thread t reads the 16-byte

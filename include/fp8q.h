@@ -90,6 +90,38 @@ int fp8q_quant_weight_128x128(const void* w_bf16, int64_t N, int64_t K, int64_t 
                               int64_t ldq, float* scales, int pow2_scale, void* stream);
 
 /*
+ * Rows and columns in one pass: the 1x128 quantization of X (exactly
+ * fp8q_quant_act_1x128) and the 1x128 quantization of X^T (128x1 tiles of X, along M)
+ * from one read of X [Q], [P2].  The transposed copy is what a Wgrad GEMM (dW = dY^T X)
+ * consumes; why-be.co.kr wr_id=57820 para 4 and why-be.co.kr wr_id=72410 para 3 describe
+ * the extra HBM round trips of quantizing and transposing in separate passes.
+ *
+ * x_bf16  device, bf16 [M, K], row stride ldx elements
+ * q, s    as fp8q_quant_act_1x128: E4M3 [M, K] (row stride ldq bytes), fp32 [K/128][ld_s >= M]
+ * qt      device, E4M3 [K, M], row stride ldqt bytes: qt[k, m] = code of x[m, k] scaled by
+ *         the amax of x[128 (m/128) .. +127, k]
+ * st      device, fp32 group-major [M/128][ld_st >= K]: st[(m/128) * ld_st + k]
+ * Requires M % 128 == 0, K % 128 == 0, ldx % 8 == 0, ldq % 8 == 0, ldqt % 16 == 0,
+ * x and qt 16-byte aligned, q 8-byte aligned.  Both outputs are bit-exact with the
+ * definition (the qt / st pair equals fp8q_quant_act_1x128 applied to X^T).
+ */
+int fp8q_quant_act_dual(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
+                        int64_t ldq, float* s, int64_t ld_s, uint8_t* qt, int64_t ldqt,
+                        float* st, int64_t ld_st, int pow2_scale, void* stream);
+
+/*
+ * Transpose of a matrix quantized in 128x128 blocks: qt = q^T (E4M3 [K, N], row stride
+ * ldqt bytes) and st = s^T (fp32 [K/128][N/128] row-major).  A block's amax is that of
+ * its transpose, so (qt, st) is exactly fp8q_quant_weight_128x128 of the transposed bf16
+ * matrix -- the B operand of a Dgrad GEMM (dX = dY W, B = W^T) -- at 2 bytes of HBM
+ * traffic per element instead of 3 for requantizing.
+ * Requires N % 128 == 0, K % 128 == 0, ldq and ldqt multiples of 16, q and qt 16-byte
+ * aligned.  Bit-exact.
+ */
+int fp8q_transpose_blocks(const uint8_t* q, const float* s, int64_t N, int64_t K, int64_t ldq,
+                          uint8_t* qt, float* st, int64_t ldqt, void* stream);
+
+/*
  * 1xK row quantization: one scale per row over all of K (the per-row baseline of the
  * accumulation study [K]; not part of the fine-grained path).  scales: device fp32 [M].
  * Requires K % 128 == 0 and the alignment of fp8q_quant_act_1x128.

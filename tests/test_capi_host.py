@@ -69,6 +69,25 @@ def test_quant_act_validation(L):
     assert f(P16, 4, 128, 132, P16, 128, P16, 4, 0, NULL) == 3          # ldx % 8
 
 
+def test_quant_dual_validation(L):
+    f = L.fp8q_quant_act_dual
+
+    def call(M=256, K=256, ldx=256, q=P16, ldq=256, s=P16, ld_s=256, qt=P16, ldqt=256, st=P16,
+             ld_st=256, x=P16):
+        return f(x, M, K, ldx, q, ldq, s, ld_s, qt, ldqt, st, ld_st, 0, NULL)
+
+    assert call(M=0) == 0                       # empty: no-op
+    assert call(M=-1) == 2
+    assert call(qt=NULL) == 1
+    assert call(M=200, ld_s=256, ldqt=256) == 2  # M % 128: the transposed K
+    assert call(K=200) == 2
+    assert call(ldqt=128) == 2                  # ldqt < M
+    assert call(ld_st=128) == 2                 # ld_st < K
+    assert call(ldqt=264) == 3                  # 16-byte row starts of qt
+    assert call(qt=P_MIS) == 3
+    assert call(x=P_MIS) == 3
+
+
 def test_quant_weight_validation(L):
     f = L.fp8q_quant_weight_128x128
     assert f(P16, 0, 128, 128, P16, 128, P16, 0, NULL) == 0

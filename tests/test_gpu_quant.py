@@ -136,3 +136,46 @@ def test_rowwise(fq):
         q_ref, s_ref = oracle.quant_rowwise(bits, pow2)
         assert_bytes_equal("rowwise.q", host(q), q_ref)
         assert_bytes_equal("rowwise.s", host(s), s_ref)
+
+
+# ---------------------------------------------------------- rows and columns in one pass
+
+def _dual_parity(fq, bits, pow2, name="dual"):
+    """Both outputs bit-exact: (q, s) with the 1x128 quantization of X, (qt, st) with the
+    1x128 quantization of X^T (the definition of the transposed copy)."""
+    q, s, qt, st = fq.quant_act_dual(to_dev_bf16(bits), pow2)
+    q_ref, s_ref = oracle.quant_act_1x128(bits, pow2)
+    qt_ref, st_ref = oracle.quant_act_1x128(np.ascontiguousarray(bits.T), pow2)
+    assert_bytes_equal(name + ".q", host(q), q_ref)
+    assert_bytes_equal(name + ".s", host(s), s_ref)
+    assert_bytes_equal(name + ".qt", host(qt), qt_ref)
+    assert_bytes_equal(name + ".st", host(st), st_ref)
+    assert fq.device_error() == 0
+
+
+@pytest.mark.parametrize("M,K", [(128, 128), (256, 384), (384, 1024), (1024, 256)])
+@pytest.mark.parametrize("pow2", [False, True])
+def test_dual_shapes(fq, M, K, pow2):
+    rng = np.random.default_rng(M * 3 + K)
+    _dual_parity(fq, workloads.normal_bf16(rng, (M, K), 1.0, 0.001), pow2, f"dual {M}x{K}")
+
+
+def test_dual_edge_tiles(fq):
+    """Zero, signed-zero and single-value columns, tiny magnitudes (subnormal scales),
+    one huge outlier per column tile."""
+    rng = np.random.default_rng(17)
+    x = workloads.bf16_bits_to_fp32(workloads.normal_bf16(rng, (256, 256), 1.0)).copy()
+    x[:128, :128] = 0.0
+    x[:128, 5] = -0.0
+    x[:128, 7] = 0.0
+    x[3, 7] = 3.0
+    x[128:, :128] *= np.float32(1e-38)
+    x[128:, 200] = 1e30
+    for pow2 in (False, True):
+        _dual_parity(fq, workloads.fp32_to_bf16_bits(x), pow2, "dual edges")
+
+
+def test_dual_dense_activation_full(fq):
+    """The dense workload's A [4096, 7168] (power-of-two scales): both copies in full."""
+    w = workloads.dense()
+    _dual_parity(fq, w.gen_a(), True, "dual dense A")

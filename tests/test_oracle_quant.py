@@ -180,3 +180,12 @@ def test_rowwise_invariants(orc):
     q1, s1 = orc.quant_rowwise(x[:, :128])
     qa, sa = orc.quant_act_1x128(x[:, :128], False)
     assert np.array_equal(q1, qa) and np.array_equal(s1, sa[0])
+
+
+def test_weight_blocks_are_symmetric_under_transposition(orc):
+    """A 128x128 block's amax is that of its transpose: quantizing W^T gives the transposed
+    codes and scales of W (the Dgrad operand needs no requantization)."""
+    w = workloads.normal_bf16(np.random.default_rng(31), (256, 384), 0.02, 0.001)
+    q, s = orc.quant_weight_128x128(w, False)
+    qt, st = orc.quant_weight_128x128(np.ascontiguousarray(w.T), False)
+    assert np.array_equal(qt, q.T) and np.array_equal(st, s.T)
