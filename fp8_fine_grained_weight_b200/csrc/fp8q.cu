@@ -39,12 +39,20 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
+// The tensor-map encoder is a driver call and needs the device's context current on the
+// calling thread.  A thread that has made no runtime call yet (a framework's worker
+// thread, say) may have none bound: make the current device's primary context current.
+bool bind_current_context() {
+  int dev = 0;
+  return cudaGetDevice(&dev) == cudaSuccess && cudaSetDevice(dev) == cudaSuccess;
+}
+
 // 2D K-major E4M3 operand: [rows, K] with a row stride of `ld` bytes; box = 128 bytes of K
 // by `box_rows` rows, 128-byte swizzle (the canonical layout the MMA descriptors expect).
 int encode_operand(CUtensorMap* tm, const void* base, uint64_t K, uint64_t rows, uint64_t ld,
                    uint32_t box_rows) {
   auto enc = tensor_map_encoder();
-  if (!enc) return FP8Q_ERR_CUDA;
+  if (!enc || !bind_current_context()) return FP8Q_ERR_CUDA;
   cuuint64_t dims[2] = {K, rows};
   cuuint64_t strides[1] = {ld};
   cuuint32_t box[2] = {128, box_rows};

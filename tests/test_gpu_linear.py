@@ -96,3 +96,40 @@ def test_fp8_linear_tracks_the_bf16_layer(fq):
     assert rel(y, yf) < 0.06
     assert rel(x.grad, xf.grad) < 0.06
     assert rel(layer.weight.grad, wf.grad) < 0.06
+
+
+def test_entry_points_on_a_fresh_thread(fq):
+    """A thread that has made no CUDA call yet (as a framework's backward worker thread may
+    be) can call the entry points that encode TMA descriptors: the library binds the
+    device's context itself."""
+    import threading
+    import torch
+    rng = np.random.default_rng(41)
+    x_bits = workloads.normal_bf16(rng, (256, 256), 1.0)
+    w_bits = workloads.normal_bf16(rng, (256, 256), 0.02)
+    x, w = to_dev_bf16(x_bits), to_dev_bf16(w_bits)
+    q, s = fq.quant_act_1x128(x, True)
+    qw, sw = fq.quant_weight_128x128(w, True)
+    torch.cuda.synchronize()
+    out, err = {}, []
+
+    def work():
+        try:   # the GEMMs (which encode TMA descriptors) are this thread's first CUDA calls
+            out["c"] = fq.gemm_blockscaled_ue8m0(q, s, qw, sw)
+            out["c2"] = fq.gemm_blockscaled(q, s, qw, sw)
+            out["qt"] = fq.quant_act_dual(x, True)[2]
+            torch.cuda.synchronize()
+        except Exception as e:                    # reported below, on the test's thread
+            err.append(e)
+
+    t = threading.Thread(target=work)
+    t.start()
+    t.join()
+    assert not err, err
+    qt_ref, _ = oracle.quant_act_1x128(np.ascontiguousarray(x_bits.T), True)
+    assert_bytes_equal("fresh-thread qt", host(out["qt"]), qt_ref)
+    qa, sa = oracle.quant_act_1x128(x_bits, True)
+    qb, sb = oracle.quant_weight_128x128(w_bits, True)
+    C, Tm = oracle.gemm_blockscaled_ref(qa, sa, qb, sb)
+    assert_gemm_close("fresh-thread ue8m0", host(out["c"]), C, Tm, bf16=True)
+    assert_gemm_close("fresh-thread promoted", host(out["c2"]), C, Tm, bf16=True)
