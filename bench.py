@@ -122,13 +122,23 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest of the ranks' values (a collective: every rank calls it)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def bench_config(w, world: int) -> dict:
+    """The `config` object of the bench line (both arms)."""
+    return {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "pow2_scales": bool(w.pow2_a and w.pow2_b),
+            "out": "fp32" if w.out_fp32 else "bf16",
+            "parallelism": f"replicas x{world} (dense: each GPU its own {w.M}-token batch)",
+            "l2": "flush between steps (512 MB write, then read back), outside the per-step events"}
 
 
 # ------------------------------------------------------------------------------ GPU arm
@@ -246,10 +256,7 @@ def run_gpu(args, rank, world):
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3 x e4m3 -> f32 accumulate, bf16 out", "data": "synthetic",
-        "config": {"workload": w.name, "M": M, "N": N, "K": K, "pow2_scales": True,
-                   "out": "bf16" if not w.out_fp32 else "fp32",
-                   "parallelism": f"replicas x{world} (dense: each GPU its own 4096-token batch)",
-                   "l2": "flush between steps (512 MB write, then read back), outside the per-step events"},
+        "config": bench_config(w, world),
         "kernels_ms": {"quant_act_1x128": round(ms_act, 5), "quant_weight_128x128": round(ms_w, 5),
                        kernel: round(ms_gemm, 5)},
         "gemm_path": path,
@@ -604,7 +611,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(dt * 1e3, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64 (oracle)", "data": "synthetic",
-            "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K},
+            "config": bench_config(w, 1),
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": os.cpu_count(),
                              "kind": "oracle",
                              "sample": f"per step: 8 rows x 128 columns x K={w.K} of the workload "
