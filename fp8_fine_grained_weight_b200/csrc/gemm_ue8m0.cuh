@@ -18,20 +18,25 @@
 // with scale 1.
 //
 // Tiles of 128 x 224 (224 divides 7168; two 224-column FP32 accumulators and the scale
-// region fill the 512 TMEM columns), persistent CTAs, 16 warps:
+// region fill the 512 TMEM columns), persistent CTAs, 12 warps:
 //   warp 0       TMA producer: A [128 x 128 B] and B [224 x 128 B] per K-group into a
 //                5-stage ring (128-byte swizzle).
-//   warp 1       TMEM owner and MMA issuer: per group 4 x block-scaled MMA (K = 32) into
-//                the tile's accumulator buffer; commits free smem stages and scale slots
-//                and publish finished tiles.
-//   warps 2-3    idle.
-//   warps 4-7    scale producers, one per 32-lane TMEM sub-partition: for 4 consecutive
-//                groups at a time, convert the FP32 scales to UE8M0 bytes (byte j of a
-//                32-bit cell = group j of the four) and store them into a scale slot:
-//                A: row m at lane m, column slot + m / 32;
-//                B: row n at column slot + 4 + n / 32, lane n % 32 of every
-//                sub-partition (each keeps its own copy).
-//   warps 8-15   epilogue: warp w drains TMEM lanes 32*(w%4).. and 112 of the 224
+//   warp 1       TMEM owner and MMA issuer.  Per slot of four groups it copies the slot's
+//                scale words from shared memory into TMEM (tcgen05.cp 32x128b.warpx4: a
+//                32-row x 16-byte block into 4 columns of every 32-lane sub-partition),
+//                then issues the groups' block-scaled MMAs (K = 32 each).  tcgen05.cp and
+//                tcgen05.mma of one thread run in issue order, so a scale slot in TMEM is
+//                rewritten only after the MMAs that read it.  Commits free smem stages,
+//                scale slots and finished accumulators.
+//   warp 2       scale producer.  For a slot (groups 4k .. 4k+3 of one tile) lane l packs
+//                the UE8M0 bytes of A rows l, 32+l, 64+l, 96+l (byte j = group 4k+j) into
+//                one 16-byte row of the A block, and those of B rows l + 32j (j < 7) into
+//                two 16-byte rows of the B blocks, in a 3-slot shared-memory ring.  After
+//                the copies the MMA reads, for A row m, lane m and column m/32, and for B
+//                row n, column 4 + n/32 and lane n % 32 of its own sub-partition: the
+//                layout of kind::mxf8f6f4 scale factors (checked on B200 with probes).
+//   warp 3       idle.
+//   warps 4-11   epilogue: warp w drains TMEM lanes 32*(w%4).. and 112 of the 224
 //                columns of a finished accumulator, converts and stores C, and frees the
 //                buffer for the tile after next.
 #pragma once
@@ -51,30 +56,53 @@ struct Ue8m0Cfg {
   static constexpr int kN = 224;                  // tile columns = MMA N
   static constexpr int kStages = 5;
   static constexpr int kAccCols = 2 * kN;         // two accumulator buffers
-  static constexpr int kSfSlots = 4;              // scale slots, 4 groups each
-  static constexpr int kSfSlotCols = 16;          // A: 4 columns, B: 7, padding: 5
+  static constexpr int kSfSmemSlots = 3;          // scale slots in shared memory, 4 groups each
+  static constexpr int kSfTmemSlots = 4;          // scale slots in TMEM
+  static constexpr int kSfSlotCols = 12;          // A: 4 columns, B: 8
   static constexpr int kSfCol0 = kAccCols;        // first scale column
-  static constexpr int kEpiWarp0 = 8, kEpiWarps = 8, kSfWarp0 = 4;
+  static constexpr int kSfWarp = 2, kEpiWarp0 = 4, kEpiWarps = 8;
   static constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
   static constexpr int kSetCols = kN / 2;         // columns per epilogue warp
   static constexpr uint32_t kABytes = 128 * kBK;
   static constexpr uint32_t kBBytes = kN * kBK;
   static constexpr uint32_t kStageTx = kABytes + kBBytes;
+  static constexpr uint32_t kSfA = 32 * 16;       // one 32 x 16 B copy block
+  static constexpr uint32_t kSfBytes = 3 * kSfA;  // A block, two B blocks
   static constexpr uint32_t a = 0;
   static constexpr uint32_t b = a + kStages * kABytes;
-  static constexpr uint32_t bars = b + kStages * kBBytes;
+  static constexpr uint32_t sf = b + kStages * kBBytes;
+  static constexpr uint32_t bars = sf + kSfSmemSlots * kSfBytes;
   // full[S], empty[S], tfull[2], tempty[2], sfull[SF], sempty[SF], drain
-  static constexpr uint32_t n_bars = 2 * kStages + 4 + 2 * kSfSlots + 1;
+  static constexpr uint32_t n_bars = 2 * kStages + 4 + 2 * kSfSmemSlots + 1;
   static constexpr uint32_t misc = align_up(bars + 8 * n_bars, 16);   // tmem slot, abort flag
   static constexpr uint32_t end = misc + 16;
   static constexpr uint32_t smem_bytes = end + 1024;
-  static_assert(kAccCols + kSfSlots * kSfSlotCols <= static_cast<int>(kTmemCols), "TMEM budget");
-  static_assert(4 + (kN + 31) / 32 <= kSfSlotCols, "scale slot holds A and B columns");
+  static_assert(kAccCols + kSfTmemSlots * kSfSlotCols <= static_cast<int>(kTmemCols), "TMEM budget");
+  static_assert((kN + 31) / 32 <= 8, "B scales fit two copy blocks");
   static_assert(kN % 16 == 0 && kN <= 256, "MMA N for M = 128");
   static_assert(kSetCols % 16 == 0, "16-column epilogue loads");
-  static_assert(kABytes % 1024 == 0 && kBBytes % 1024 == 0, "swizzle atoms");
+  static_assert(kABytes % 1024 == 0 && kBBytes % 1024 == 0 && sf % 1024 == 0, "alignment");
   static_assert(smem_bytes <= 232448, "fits the 227 KB opt-in shared memory");
 };
+
+// Shared-memory descriptor of a 32-row x 16-byte block (no swizzle: 8-row core matrices of
+// 128 bytes, stacked) for tcgen05.cp; fields as in smem_desc_k_sw128, layout 0.
+__device__ __forceinline__ uint64_t smem_desc_copy32x16(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);
+  d |= static_cast<uint64_t>(128 >> 4) << 16;
+  d |= static_cast<uint64_t>(128 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;
+}
+
+__device__ __forceinline__ void tmem_copy_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 
 // UE8M0 byte of a power-of-two FP32 scale; sets `bad` for anything else.
 __device__ __forceinline__ uint32_t ue8m0_of(float s, bool& bad) {
@@ -92,7 +120,8 @@ __global__ void __launch_bounds__(Ue8m0Cfg::kThreads, 1)
                           const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
   using Cfg = Ue8m0Cfg;
   constexpr int S = Cfg::kStages;
-  constexpr int SF = Cfg::kSfSlots;
+  constexpr int SF = Cfg::kSfSmemSlots;
+  constexpr int TS = Cfg::kSfTmemSlots;
   constexpr int kN = Cfg::kN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -122,7 +151,7 @@ __global__ void __launch_bounds__(Ue8m0Cfg::kThreads, 1)
       mbar_init(tempty_bar(b), 32 * Cfg::kEpiWarps);   // every epilogue thread
     }
     for (int r = 0; r < SF; ++r) {
-      mbar_init(sfull_bar(r), 4);                       // one arrive per scale warp
+      mbar_init(sfull_bar(r), 1);                       // the scale producer
       mbar_init(sempty_bar(r), 1);                      // the MMA thread's commit
     }
     mbar_init(drain_bar, 1);
@@ -190,10 +219,17 @@ __global__ void __launch_bounds__(Ue8m0Cfg::kThreads, 1)
         for (int g = 0; g < G; ++g, ++it) {
           const int s = it % S;
           const int r = sc % SF;
-          if ((g & 3) == 0 &&
-              !mbar_wait(sfull_bar(r), (sc / SF) & 1u, kSiteScales, abort_flag)) {
-            ok = false;
-            break;
+          const uint32_t sfa = tmem_base + Cfg::kSfCol0 + (sc % TS) * Cfg::kSfSlotCols;
+          if ((g & 3) == 0) {
+            if (!mbar_wait(sfull_bar(r), (sc / SF) & 1u, kSiteScales, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t src = sbase + Cfg::sf + r * Cfg::kSfBytes;
+            tmem_copy_32x128b_x4(sfa, smem_desc_copy32x16(src));
+            tmem_copy_32x128b_x4(sfa + 4, smem_desc_copy32x16(src + Cfg::kSfA));
+            tmem_copy_32x128b_x4(sfa + 8, smem_desc_copy32x16(src + 2 * Cfg::kSfA));
           }
           if (!mbar_wait(full_bar(s), (it / S) & 1u, kSiteMmaFull, abort_flag)) {
             ok = false;
@@ -202,14 +238,13 @@ __global__ void __launch_bounds__(Ue8m0Cfg::kThreads, 1)
           tc_fence_after();
           const uint32_t byte = static_cast<uint32_t>(g & 3);
           const uint32_t idesc = idesc_e4m3_ue8m0(Cfg::kTileM, kN, byte);
-          const uint32_t sf = tmem_base + Cfg::kSfCol0 + r * Cfg::kSfSlotCols;
-          const uint32_t sfa = sf | (byte << 30), sfb = (sf + 4) | (byte << 30);
+          const uint32_t sfa_b = sfa | (byte << 30), sfb_b = (sfa + 4) | (byte << 30);
           const uint32_t a_addr = sbase + Cfg::a + s * Cfg::kABytes;
           const uint32_t b_addr = sbase + Cfg::b + s * Cfg::kBBytes;
 #pragma unroll
           for (int kk = 0; kk < kBK / 32; ++kk)
             mma_f8_ue8m0(d, smem_desc_k_sw128(a_addr + 32 * kk), smem_desc_k_sw128(b_addr + 32 * kk),
-                         idesc, (g > 0 || kk > 0) ? 1u : 0u, sfa, sfb);
+                         idesc, (g > 0 || kk > 0) ? 1u : 0u, sfa_b, sfb_b);
           mma_commit<1>(empty_bar(s));
           if ((g & 3) == 3 || g == G - 1) {       // the slot's last group: free it when read
             mma_commit<1>(sempty_bar(r));
@@ -222,38 +257,38 @@ __global__ void __launch_bounds__(Ue8m0Cfg::kThreads, 1)
       mma_commit<1>(drain_bar);
       mbar_wait(drain_bar, 0, kSiteDrain, nullptr);
     }
-  } else if (warp >= Cfg::kSfWarp0 && warp < Cfg::kSfWarp0 + 4) {
-    // -------------------------------------------------------------- scale producers
-    // This warp's sub-partition: TMEM lanes 32*q .. 32*q + 31.  Slots hold four groups
-    // of one tile (4k .. 4k + 3; the tile's last slot may be partial); the CTA's slots
-    // run in order (tile i, slot k), and the raw scales of the next slot are loaded before
-    // the current one is stored.
-    //   A: lane l loads the 4 scales of row row0 + 32q + l.
+  } else if (warp == Cfg::kSfWarp) {
+    // -------------------------------------------------------------- scale producer
+    // Slots hold four groups of one tile (4k .. 4k + 3; a tile's last slot may be
+    // partial); the CTA's slots run in order (tile i, slot k), and the raw scales of the
+    // next slot are loaded before the current one is stored.
+    //   A: lane l loads the 4 groups' scales of rows l + 32j, j < 4.
     //   B, 128x128 blocks: the tile's 224 rows touch at most 3 blocks; lane l < 12 loads
-    //     block nb0 + l / 4, group 4k + l % 4, and the packed words are gathered by
-    //     shuffles (every 32-row chunk of the tile lies inside one block).
-    //   B, 1x128 rows: lane l loads the 4 scales of each of its 7 rows.
-    const int q = warp & 3;
-    const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+    //     block nb0 + l / 4, group 4k + l % 4, and shuffles build the packed words (every
+    //     32-row chunk of the tile lies inside one block).
+    //   B, 1x128 rows: lane l loads the 4 groups' scales of rows l + 32j, j < 7.
     constexpr int kRawB = ROW_B ? 28 : 1;
     struct Raw {
-      float a[4];
+      float a[16];
       float b[kRawB];
     };
     bool bad = false;
     auto fetch = [&](int i, int k, Raw& raw) {
 #pragma unroll
-      for (int b = 0; b < 4; ++b) raw.a[b] = 1.0f;
+      for (int j = 0; j < 16; ++j) raw.a[j] = 1.0f;
 #pragma unroll
       for (int j = 0; j < kRawB; ++j) raw.b[j] = 1.0f;
       if (i >= n_tiles) return;
       int64_t row0, col0;
       tile_of(i, row0, col0);
-      const int64_t m = row0 + 32 * q + lane;
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const int g = 4 * k + b;
-        if (g < G && m < p.M) raw.a[b] = __ldg(p.sA + static_cast<int64_t>(g) * p.ld_sa + m);
+      for (int j = 0; j < 4; ++j) {
+        const int64_t m = row0 + 32 * j + lane;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int g = 4 * k + b;
+          if (g < G && m < p.M) raw.a[4 * j + b] = __ldg(p.sA + static_cast<int64_t>(g) * p.ld_sa + m);
+        }
       }
       if (ROW_B) {
 #pragma unroll
@@ -271,24 +306,24 @@ __global__ void __launch_bounds__(Ue8m0Cfg::kThreads, 1)
         if (lane < 12 && g < G && nb * 128 < p.N) raw.b[0] = __ldg(p.sB + nb * G + g);
       }
     };
-    // Packs and stores the slot once the MMAs that read its previous contents are done.
-    // Returns false (warp-uniform) on abort or timeout.
+    // Packs the slot into its shared-memory blocks once the MMA thread has copied the
+    // ring slot's previous contents.  Returns false (warp-uniform) on abort or timeout.
     auto emit = [&](int i, int64_t sc, const Raw& raw) -> bool {
       int64_t row0, col0;
       tile_of(i, row0, col0);
-      uint32_t v[16];
-      uint32_t wa = 0;
+      uint32_t wa[4], wb[8];
 #pragma unroll
-      for (int b = 0; b < 4; ++b) wa |= ue8m0_of(raw.a[b], bad) << (8 * b);
+      for (int j = 0; j < 4; ++j) {
+        wa[j] = 0;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) v[j] = wa;            // only column q is read for these lanes
+        for (int b = 0; b < 4; ++b) wa[j] |= ue8m0_of(raw.a[4 * j + b], bad) << (8 * b);
+      }
       if (ROW_B) {
 #pragma unroll
         for (int j = 0; j < 7; ++j) {
-          uint32_t w = 0;
+          wb[j] = 0;
 #pragma unroll
-          for (int b = 0; b < 4; ++b) w |= ue8m0_of(raw.b[4 * j + b], bad) << (8 * b);
-          v[4 + j] = w;
+          for (int b = 0; b < 4; ++b) wb[j] |= ue8m0_of(raw.b[4 * j + b], bad) << (8 * b);
         }
       } else {
         const uint32_t byte = ue8m0_of(raw.b[0], bad);
@@ -303,20 +338,20 @@ __global__ void __launch_bounds__(Ue8m0Cfg::kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 7; ++j) {
           const int jb = static_cast<int>((col0 + 32 * j) / 128) - nb0;
-          v[4 + j] = jb == 0 ? w[0] : (jb == 1 ? w[1] : w[2]);
+          wb[j] = jb == 0 ? w[0] : (jb == 1 ? w[1] : w[2]);
         }
       }
-#pragma unroll
-      for (int j = 11; j < 16; ++j) v[j] = 0;
+      wb[7] = 0;
       const int r = static_cast<int>(sc % SF);
-      // warp-uniform outcome: the TMEM store below is a whole-warp instruction
+      // warp-uniform outcome (the warp writes the slot together)
       const bool got = mbar_wait(sempty_bar(r), static_cast<uint32_t>(((sc / SF) & 1) ^ 1), kSiteScales,
                                  abort_flag);
       if (!__all_sync(0xFFFFFFFFu, got)) return false;
-      tc_fence_after();
-      tmem_st_16cols(tmem_base + lane_base + Cfg::kSfCol0 + r * Cfg::kSfSlotCols, v);
-      tmem_st_wait();
-      tc_fence_before();
+      uint8_t* blk = smem + Cfg::sf + r * Cfg::kSfBytes;
+      *reinterpret_cast<uint4*>(blk + 16 * lane) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+      *reinterpret_cast<uint4*>(blk + Cfg::kSfA + 16 * lane) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+      *reinterpret_cast<uint4*>(blk + 2 * Cfg::kSfA + 16 * lane) = make_uint4(wb[4], wb[5], wb[6], wb[7]);
+      fence_proxy_async_smem();                          // visible to tcgen05.cp
       __syncwarp();
       if (lane == 0) mbar_arrive(sfull_bar(r));
       return true;
