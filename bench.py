@@ -496,6 +496,16 @@ def profile_case(args, name: str, launches: int = 3):
     """A few launches of one workload's kernels on device-drawn inputs (for ncu captures)."""
     import torch
     import fp8_fine_grained_weight_b200 as fq
+    if name == "dual":     # rows + transposed copy of a 16384-token x 7168 gradient
+        dY = _dev_normal((16384, 7168), 1e-3, 7003)
+        bufs = fq.quant_act_dual(dY, False)
+        for _ in range(launches):
+            fq.quant_act_dual(dY, False, out=bufs)
+        torch.cuda.synchronize()
+        if fq.device_error():
+            raise RuntimeError("device error word set")
+        print(json.dumps({"profile_case": "quant_act_dual_16384x7168", "launches": launches}), flush=True)
+        return
     w = workloads.ALL[name]()
     if w.experts:
         off = torch.from_numpy(w.offsets).cuda()
@@ -636,7 +646,7 @@ def main():
     ap.add_argument("--no-check", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' timings")
     ap.add_argument("--no-study", action="store_true", help="skip the accumulation study")
-    ap.add_argument("--profile-case", choices=["tiny", "dense", "prefill", "decode", "wgrad"],
+    ap.add_argument("--profile-case", choices=["tiny", "dense", "prefill", "decode", "wgrad", "dual"],
                     help="only run a few GEMM launches of one workload (for ncu) and exit")
     args = ap.parse_args()
 

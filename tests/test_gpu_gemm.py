@@ -353,6 +353,15 @@ def test_ue8m0_rowwise_b_scales(fq, M, N, K):
     _dense_case(fq, a, b, True, True, True, b_rowwise=True, name="ue8m0 row-b", ue8m0=True)
 
 
+def test_ue8m0_long_k_rowwise(fq):
+    """K = 16384 (128 groups, 32 scale slots per tile) with 1x128 scales on both operands,
+    the wgrad shape at 512 x 640; all rows against the oracle."""
+    rng = np.random.default_rng(77)
+    a = _spread_scales(rng, workloads.normal_bf16(rng, (512, 16384), 1e-3), 1, span=6)
+    b = workloads.normal_bf16(rng, (640, 16384), 1.0)
+    _dense_case(fq, a, b, True, True, True, b_rowwise=True, name="ue8m0 long K", ue8m0=True)
+
+
 def test_ue8m0_dense_full_size_sampled_rows(fq):
     """The dense workload (power-of-two scales) at full size through the tensor-core-scaled
     GEMM; 96 sampled rows spanning every M tile and the last row."""
