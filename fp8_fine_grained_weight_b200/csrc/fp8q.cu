@@ -63,19 +63,14 @@ int encode_operand(CUtensorMap* tm, const void* base, uint64_t K, uint64_t rows,
   return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
-// Tile shapes.  Promotion every 128 K hands each TMEM accumulator from the tensor core to
-// the epilogue warps and back once per K-group.  The kernel template has two shapes:
-//  * single CTA, 128 x 256 tiles: 2 accumulator buffers of 256 columns;
-//  * CTA pair (cta_group::2), 256 x 128 tiles: 4 buffers of 128 columns per CTA, each CTA
-//    loading 128 rows of A and 64 of B per stage.
-// Both pass the same parity tests.  On B200 the pair is the slower of the two for every
-// promoted workload measured (dense 4096 x 7168 x 7168: 0.34 ms against 0.24 ms): its
-// groups are half as large, and the per-group cost of the hand-off (barrier waits, two
-// TMEM loads per epilogue warp, the release) is paid twice as often.  The launcher
-// therefore uses the single-CTA tiles; the pair instantiation is kept for the shapes
-// where that balance changes.
-bool dense_pair(int64_t) { return false; }
-bool grouped_pair(int64_t, int) { return false; }
+// Tile shape of the promoted GEMMs: one CTA per 128 x 256 tile, two 256-column TMEM
+// accumulator buffers.  The kernel template also has a CTA-pair shape (cta_group::2,
+// 256 x 128 tiles, four 128-column buffers per CTA); it passed the same parity tests but
+// measured slower on every promoted workload (dense 4096 x 7168 x 7168: 0.34 ms against
+// 0.24 ms: its groups are half as large, so the per-group hand-off is paid twice as
+// often), and the launcher does not instantiate it.
+constexpr bool kPair = false;
+using Cfg1 = fp8q::GemmCfg<kPair>;
 
 template <bool PAIR, bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16>
 struct GemmLauncher {
@@ -115,7 +110,10 @@ struct GemmLauncher {
     config(cfg, attr, nullptr);
     cfg.gridDim = dim3(static_cast<unsigned>(sms / Cfg::kCG * Cfg::kCG));
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) n = sms / Cfg::kCG;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+      (void)cudaGetLastError();   // the query's failure is handled here, not by the next launch check
+      n = sms / Cfg::kCG;
+    }
     cached[dev].store(n, std::memory_order_release);
     return n;
   }
@@ -458,20 +456,17 @@ int fp8_gemm_blockscaled_ws(const uint8_t* A, const float* sA, int64_t ld_sa, co
   if (b_scale_mode == FP8Q_BSCALE_ROW1x128 && ld_sb < N) return FP8Q_ERR_SHAPE;
   if (!aligned(sA, 4) || !aligned(sB, 4)) return FP8Q_ERR_ALIGN;
   if (workspace != nullptr && !aligned(workspace, 16)) return FP8Q_ERR_ALIGN;
-  const bool pair = dense_pair(M);
   CUtensorMap tmA, tmB;
   if ((st = encode_operand(&tmA, A, K, M, lda, 128)) != FP8Q_OK) return st;
-  const uint32_t b_rows = pair ? fp8q::GemmCfg<true>::kBRows : fp8q::GemmCfg<false>::kBRows;
-  if ((st = encode_operand(&tmB, B, K, N, ldb, b_rows)) != FP8Q_OK) return st;
+  if ((st = encode_operand(&tmB, B, K, N, ldb, Cfg1::kBRows)) != FP8Q_OK) return st;
   GemmArgs a{};
   a.sA = sA; a.ld_sa = ld_sa; a.sB = sB; a.ld_sb = ld_sb; a.C = C; a.ldc = ldc;
   a.M = M; a.N = N; a.G = static_cast<int>(K / 128); a.m_offsets = nullptr; a.num_experts = 0;
-  const int64_t tiles = pair ? dense_tiles<true>(M, N) : dense_tiles<false>(M, N);
+  const int64_t tiles = dense_tiles<kPair>(M, N);
   if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   const bool row_b = b_scale_mode == FP8Q_BSCALE_ROW1x128, bf16 = out_dtype == FP8Q_OUT_BF16;
-  const auto s = static_cast<cudaStream_t>(stream);
-  return pair ? dispatch_dense<true>(tmA, tmB, a, row_b, bf16, tiles, workspace, workspace_bytes, s)
-              : dispatch_dense<false>(tmA, tmB, a, row_b, bf16, tiles, workspace, workspace_bytes, s);
+  return dispatch_dense<kPair>(tmA, tmB, a, row_b, bf16, tiles, workspace, workspace_bytes,
+                               static_cast<cudaStream_t>(stream));
 }
 
 int fp8_gemm_blockscaled(const uint8_t* A, const float* sA, int64_t ld_sa, const uint8_t* B,
@@ -519,17 +514,10 @@ int fp8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, size_t* bytes) {
   if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_SHAPE;
   if (M == 0 || N == 0 || K == 0) return FP8Q_OK;
   if (K % 128 != 0 || N % 128 != 0) return FP8Q_ERR_SHAPE;
-  // The plan of the tile shape fp8_gemm_blockscaled_ws will choose for M; both B scale
-  // modes and output types share it.
-  if (dense_pair(M)) {
-    const int units = GemmLauncher<true, true, false, false, true>::max_units();
-    if (units <= 0) return FP8Q_ERR_CUDA;
-    *bytes = plan_split<true>(dense_tiles<true>(M, N), K / 128, units).ws_bytes;
-  } else {
-    const int units = GemmLauncher<false, true, false, false, true>::max_units();
-    if (units <= 0) return FP8Q_ERR_CUDA;
-    *bytes = plan_split<false>(dense_tiles<false>(M, N), K / 128, units).ws_bytes;
-  }
+  // both B scale modes and output types share the plan
+  const int units = GemmLauncher<kPair, true, false, false, true>::max_units();
+  if (units <= 0) return FP8Q_ERR_CUDA;
+  *bytes = plan_split<kPair>(dense_tiles<kPair>(M, N), K / 128, units).ws_bytes;
   return FP8Q_OK;
 }
 
@@ -545,27 +533,22 @@ int fp8_gemm_grouped(const uint8_t* A, const float* sA, int64_t ld_sa, const uin
   if (ld_sa < max_sum_M) return FP8Q_ERR_SHAPE;
   if (!aligned(sA, 4) || !aligned(sW, 4) || !aligned(m_offsets, 4)) return FP8Q_ERR_ALIGN;
   if (static_cast<int64_t>(num_groups) * N > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  const bool pair = grouped_pair(max_sum_M, num_groups);
   CUtensorMap tmA, tmB;
   if ((st = encode_operand(&tmA, A, K, max_sum_M, K, 128)) != FP8Q_OK) return st;
-  const uint32_t b_rows = pair ? fp8q::GemmCfg<true>::kBRows : fp8q::GemmCfg<false>::kBRows;
-  if ((st = encode_operand(&tmB, W, K, static_cast<uint64_t>(num_groups) * N, K, b_rows)) != FP8Q_OK)
+  if ((st = encode_operand(&tmB, W, K, static_cast<uint64_t>(num_groups) * N, K, Cfg1::kBRows)) !=
+      FP8Q_OK)
     return st;
   GemmArgs a{};
   a.sA = sA; a.ld_sa = ld_sa; a.sB = sW; a.ld_sb = 0; a.C = C; a.ldc = N;
   a.M = max_sum_M; a.N = N; a.G = static_cast<int>(K / 128);
   a.m_offsets = m_offsets; a.num_experts = num_groups;
   // Upper bound on tiles (every group may add one partial m-tile) sizes the persistent grid.
-  const int64_t tile_m = pair ? fp8q::GemmCfg<true>::kTileM : fp8q::GemmCfg<false>::kTileM;
-  const int64_t tile_n = pair ? fp8q::GemmCfg<true>::kN : fp8q::GemmCfg<false>::kN;
-  const int64_t bound = ((max_sum_M + tile_m - 1) / tile_m + num_groups) * ((N + tile_n - 1) / tile_n);
+  const int64_t bound = ((max_sum_M + Cfg1::kTileM - 1) / Cfg1::kTileM + num_groups) *
+                        ((N + Cfg1::kN - 1) / Cfg1::kN);
   if (bound > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   const auto s = static_cast<cudaStream_t>(stream);
-  if (out_dtype == FP8Q_OUT_BF16)
-    return pair ? run_gemm<true, true, false, true, true>(tmA, tmB, a, bound, nullptr, 0, s)
-                : run_gemm<false, true, false, true, true>(tmA, tmB, a, bound, nullptr, 0, s);
-  return pair ? run_gemm<true, true, false, true, false>(tmA, tmB, a, bound, nullptr, 0, s)
-              : run_gemm<false, true, false, true, false>(tmA, tmB, a, bound, nullptr, 0, s);
+  if (out_dtype == FP8Q_OUT_BF16) return run_gemm<kPair, true, false, true, true>(tmA, tmB, a, bound, nullptr, 0, s);
+  return run_gemm<kPair, true, false, true, false>(tmA, tmB, a, bound, nullptr, 0, s);
 }
 
 int fp8_gemm_nopromo(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB, float* C,
