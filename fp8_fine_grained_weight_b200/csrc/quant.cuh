@@ -208,9 +208,11 @@ __global__ void __launch_bounds__(256) quant_act_1x128_kernel(const uint16_t* __
 //   q  / s : the 1x128 quantization of X (along K; for Fprop and Dgrad), and
 //   qt / st: the 1x128 quantization of X^T (along M, i.e. 128x1 tiles of X; for Wgrad),
 // qt [K, M] with row stride ldqt, st group-major [M/128][ldst].  why-be.co.kr wr_id=57820
-// para 4 and why-be.co.kr wr_id=72410 para 3 note that the quantization pass reads the
-// activations from HBM and that the transposed copy needed by the backward pass costs
-// another round trip; this kernel reads each element once for both.
+// para 4 describes the HBM round trip of the quantization pass (128 bf16 values read,
+// FP8 written back, read again by the MMA); why-be.co.kr wr_id=72410 para 3 asks for
+// support of transposed GEMM operations (the section's text is cut off in the pages).
+// The Wgrad GEMM consumes the transposed copy; this kernel reads each element once for
+// both copies.
 //
 // Grid (M/128, K/128), 256 threads, one 128x128 tile of X per block:
 //  rows:    as quant_act_1x128_kernel (teams of 4 lanes per row, 16 rows per warp), all

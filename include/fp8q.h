@@ -93,8 +93,9 @@ int fp8q_quant_weight_128x128(const void* w_bf16, int64_t N, int64_t K, int64_t 
  * Rows and columns in one pass: the 1x128 quantization of X (exactly
  * fp8q_quant_act_1x128) and the 1x128 quantization of X^T (128x1 tiles of X, along M)
  * from one read of X [Q], [P2].  The transposed copy is what a Wgrad GEMM (dW = dY^T X)
- * consumes; why-be.co.kr wr_id=57820 para 4 and why-be.co.kr wr_id=72410 para 3 describe
- * the extra HBM round trips of quantizing and transposing in separate passes.
+ * consumes.  why-be.co.kr wr_id=57820 para 4 describes the HBM round trip of the
+ * quantization pass; why-be.co.kr wr_id=72410 para 3 asks for support of transposed GEMM
+ * operations (its text is cut off in the pages); one read serves both copies here.
  *
  * x_bf16  device, bf16 [M, K], row stride ldx elements
  * q, s    as fp8q_quant_act_1x128: E4M3 [M, K] (row stride ldq bytes), fp32 [K/128][ld_s >= M]
