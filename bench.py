@@ -377,6 +377,14 @@ def config_throughput(fq, flush_l2, reps=10):
         "gemm_ms": round(t_g, 4), "gemm_tflops": round(tf, 1), "gemm_frac_of_fp8_peak": round(tf / fp8_peak, 4),
         "quant_act_gbs": round(w.M * w.K * (3 + 4 / 128) / (t_a * 1e-3) / 1e9, 1),
         "quant_weight_gbs": round(W.numel() * (3 + 4 / 16384) / (t_w * 1e-3) / 1e9, 1)}
+    # the same shapes with power-of-two scales on both operands, scaled in the tensor core
+    qA, sA = fq.quant_act_1x128(A, True, out=(qA, sA))
+    qW, sW = fq.quant_weight_128x128(W, True, out=(qW, sW))
+    t_u = _time_ms(lambda: fq.gemm_grouped_ue8m0(qA, sA, qW, sW, off, out=C), reps, flush_l2)
+    tf_u = w.gemm_flops / (t_u * 1e-3) / 1e12
+    out["moe_prefill_pow2_ue8m0"] = {"workload": w.name + " (power-of-two scales)", "gemm_ms": round(t_u, 4),
+                                     "gemm_tflops": round(tf_u, 1),
+                                     "gemm_frac_of_fp8_peak": round(tf_u / fp8_peak, 4)}
     del A, W, qA, sA, qW, sW, C
     # MoE decode: 64 experts, M_e ~ U{1..256}, W [7168, 2048] already FP8
     w = workloads.decode()
@@ -394,6 +402,13 @@ def config_throughput(fq, flush_l2, reps=10):
         "gemm_gbs": round(gemm_bytes / (t_g * 1e-3) / 1e9, 1),
         "gemm_frac_of_hbm": round(gemm_bytes / (t_g * 1e-3) / 1e9 / hbm, 4),
         "algorithmic_bytes": int(gemm_bytes)}
+    # the same with power-of-two weight scales too, scaled in the tensor core
+    qW, sW = fq.quant_weight_128x128(W, True, out=(qW, sW))
+    t_u = _time_ms(lambda: fq.gemm_grouped_ue8m0(qA, sA, qW, sW, off, out=C), reps, flush_l2)
+    out["moe_decode_pow2w_ue8m0"] = {
+        "workload": w.name + " (power-of-two weight scales too)", "gemm_ms": round(t_u, 4),
+        "gemm_gbs": round(gemm_bytes / (t_u * 1e-3) / 1e9, 1),
+        "gemm_frac_of_hbm": round(gemm_bytes / (t_u * 1e-3) / 1e9 / hbm, 4)}
     del A, W, qA, sA, qW, sW, C
     # wgrad: dY [7168, 16384] x X [2048, 16384], 1x128 both, fp32 out
     w = workloads.wgrad()

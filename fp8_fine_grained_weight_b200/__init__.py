@@ -42,6 +42,8 @@ SIGNATURES = {
                                     _i64, _i64, _i64, _i64, _i64, _i64, _vp]),
     "fp8_gemm_blockscaled_ue8m0": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _i32, _vp, _i32,
                                           _i64, _i64, _i64, _i64, _i64, _i64, _vp]),
+    "fp8_gemm_grouped_ue8m0": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _i32, _vp, _i32, _i64, _i64,
+                                      _i64, _vp]),
     "fp8_gemm_blockscaled_ws": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _i32, _vp, _i32,
                                        _i64, _i64, _i64, _i64, _i64, _i64, _vp, ctypes.c_size_t, _vp]),
     "fp8_gemm_workspace_size": (_i32, [_i64, _i64, _i64, ctypes.POINTER(ctypes.c_size_t)]),
@@ -292,10 +294,10 @@ def gemm_blockscaled_ue8m0(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor,
     return out
 
 
-def gemm_grouped(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor,
+def _gemm_grouped(entry: str, qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor,
                  m_offsets: torch.Tensor, out_dtype=torch.bfloat16,
                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """MoE grouped GEMM: rows m_offsets[e]..m_offsets[e+1] of A times W[e]^T.
+    """MoE grouped GEMM through `entry`: rows m_offsets[e]..m_offsets[e+1] of A times W[e]^T.
 
     qa uint8 [sumM, K]; sa fp32 [K/128, >= sumM]; qw uint8 [E, N, K]; sw fp32 [E, N/128, K/128];
     m_offsets int32 [E + 1] on the device (read by the kernel, no host sync).
@@ -314,10 +316,26 @@ def gemm_grouped(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: torch
         raise ValueError("m_offsets must have E + 1 entries")
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=qa.device)
-    _call("fp8_gemm_grouped", qa.data_ptr(), sa.data_ptr(), sa.stride(0), qw.data_ptr(),
+    _call(entry, qa.data_ptr(), sa.data_ptr(), sa.stride(0), qw.data_ptr(),
           sw.data_ptr(), out.data_ptr(), _out_code(out.dtype), m_offsets.data_ptr(), E, M, N, K,
           _stream(qa))
     return out
+
+
+def gemm_grouped(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor,
+                 m_offsets: torch.Tensor, out_dtype=torch.bfloat16,
+                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """MoE grouped GEMM with per-128-K promotion: rows m_offsets[e]..m_offsets[e+1] of A
+    times W[e]^T.  qa uint8 [sumM, K]; sa fp32 [K/128, >= sumM]; qw uint8 [E, N, K];
+    sw fp32 [E, N/128, K/128]; m_offsets int32 [E + 1] on the device."""
+    return _gemm_grouped("fp8_gemm_grouped", qa, sa, qw, sw, m_offsets, out_dtype, out)
+
+
+def gemm_grouped_ue8m0(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor,
+                       m_offsets: torch.Tensor, out_dtype=torch.bfloat16,
+                       out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """gemm_grouped for power-of-two scales, applied inside the tensor core."""
+    return _gemm_grouped("fp8_gemm_grouped_ue8m0", qa, sa, qw, sw, m_offsets, out_dtype, out)
 
 
 def gemm_nopromo(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor,

@@ -226,11 +226,11 @@ static_assert(fp8q::kErrScale == FP8Q_ERR_SCALE, "device status code of a bad sc
 
 // Launch of the power-of-two-scale GEMM: one persistent CTA per SM (kernel attributes set
 // and the co-resident count cached per device on first use).
-template <bool ROW_B, bool OUT_BF16>
+template <bool ROW_B, bool OUT_BF16, bool GROUPED>
 int run_gemm_ue8m0(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
                    int64_t tiles, cudaStream_t st) {
-  using Cfg = fp8q::Ue8m0Cfg;
-  static constexpr auto kern = fp8q::gemm_fp8_ue8m0_kernel<ROW_B, OUT_BF16>;
+  using Cfg = fp8q::Ue8m0Cfg<GROUPED>;
+  static constexpr auto kern = fp8q::gemm_fp8_ue8m0_kernel<ROW_B, OUT_BF16, GROUPED>;
   static std::atomic<int> cached[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8Q_ERR_CUDA;
@@ -481,7 +481,7 @@ int fp8_gemm_blockscaled_ue8m0(const uint8_t* A, const float* sA, int64_t ld_sa,
                                const uint8_t* B, const float* sB, int64_t ld_sb, int b_scale_mode,
                                void* C, int out_dtype, int64_t M, int64_t N, int64_t K,
                                int64_t lda, int64_t ldb, int64_t ldc, void* stream) {
-  using Cfg = fp8q::Ue8m0Cfg;
+  using Cfg = fp8q::Ue8m0Cfg<false>;
   if (M == 0 && N >= 0 && K >= 0) return FP8Q_OK;
   int st = check_gemm_common(A, B, C, out_dtype, M, N, K, lda, ldb, ldc);
   if (st != FP8Q_OK) return st;
@@ -502,10 +502,40 @@ int fp8_gemm_blockscaled_ue8m0(const uint8_t* A, const float* sA, int64_t ld_sa,
   const auto s = static_cast<cudaStream_t>(stream);
   const bool row_b = b_scale_mode == FP8Q_BSCALE_ROW1x128;
   if (out_dtype == FP8Q_OUT_BF16)
-    return row_b ? run_gemm_ue8m0<true, true>(tmA, tmB, a, tiles, s)
-                 : run_gemm_ue8m0<false, true>(tmA, tmB, a, tiles, s);
-  return row_b ? run_gemm_ue8m0<true, false>(tmA, tmB, a, tiles, s)
-               : run_gemm_ue8m0<false, false>(tmA, tmB, a, tiles, s);
+    return row_b ? run_gemm_ue8m0<true, true, false>(tmA, tmB, a, tiles, s)
+                 : run_gemm_ue8m0<false, true, false>(tmA, tmB, a, tiles, s);
+  return row_b ? run_gemm_ue8m0<true, false, false>(tmA, tmB, a, tiles, s)
+               : run_gemm_ue8m0<false, false, false>(tmA, tmB, a, tiles, s);
+}
+
+int fp8_gemm_grouped_ue8m0(const uint8_t* A, const float* sA, int64_t ld_sa, const uint8_t* W,
+                           const float* sW, void* C, int out_dtype, const int32_t* m_offsets,
+                           int num_groups, int64_t max_sum_M, int64_t N, int64_t K, void* stream) {
+  using Cfg = fp8q::Ue8m0Cfg<true>;
+  if (max_sum_M < 0 || N < 0 || K < 0) return FP8Q_ERR_SHAPE;
+  if (num_groups < 1 || num_groups > fp8q::kMaxGroups) return FP8Q_ERR_UNSUPPORTED;
+  if (max_sum_M == 0) return FP8Q_OK;
+  int st = check_gemm_common(A, W, C, out_dtype, max_sum_M, N, K, K, K, N);
+  if (st != FP8Q_OK) return st;
+  if (!sA || !sW || !m_offsets) return FP8Q_ERR_NULL;
+  if (ld_sa < max_sum_M) return FP8Q_ERR_SHAPE;
+  if (!aligned(sA, 4) || !aligned(sW, 4) || !aligned(m_offsets, 4)) return FP8Q_ERR_ALIGN;
+  if (static_cast<int64_t>(num_groups) * N > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
+  CUtensorMap tmA, tmB;
+  if ((st = encode_operand(&tmA, A, K, max_sum_M, K, Cfg::kTileM)) != FP8Q_OK) return st;
+  if ((st = encode_operand(&tmB, W, K, static_cast<uint64_t>(num_groups) * N, K, Cfg::kN)) != FP8Q_OK)
+    return st;
+  GemmArgs a{};
+  a.sA = sA; a.ld_sa = ld_sa; a.sB = sW; a.ld_sb = 0; a.C = C; a.ldc = N;
+  a.M = max_sum_M; a.N = N; a.G = static_cast<int>(K / 128);
+  a.m_offsets = m_offsets; a.num_experts = num_groups;
+  // Upper bound on tiles (every group may add one partial m-tile) sizes the persistent grid.
+  const int64_t bound = ((max_sum_M + Cfg::kTileM - 1) / Cfg::kTileM + num_groups) *
+                        ((N + Cfg::kN - 1) / Cfg::kN);
+  if (bound > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
+  const auto s = static_cast<cudaStream_t>(stream);
+  return out_dtype == FP8Q_OUT_BF16 ? run_gemm_ue8m0<false, true, true>(tmA, tmB, a, bound, s)
+                                    : run_gemm_ue8m0<false, false, true>(tmA, tmB, a, bound, s);
 }
 
 int fp8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, size_t* bytes) {

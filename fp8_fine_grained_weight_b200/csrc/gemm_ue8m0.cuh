@@ -51,10 +51,11 @@ namespace fp8q {
 constexpr unsigned int kSiteScaleFormat = 8;
 constexpr unsigned int kErrScale = 7;            // FP8Q_ERR_SCALE
 
+template <bool GROUPED>
 struct Ue8m0Cfg {
   static constexpr int kTileM = 128;
   static constexpr int kN = 224;                  // tile columns = MMA N
-  static constexpr int kStages = 5;
+  static constexpr int kStages = GROUPED ? 4 : 5; // grouped: room for the tile table
   static constexpr int kAccCols = 2 * kN;         // two accumulator buffers
   static constexpr int kSfSmemSlots = 3;          // scale slots in shared memory, 4 groups each
   static constexpr int kSfTmemSlots = 4;          // scale slots in TMEM
@@ -75,7 +76,8 @@ struct Ue8m0Cfg {
   // full[S], empty[S], tfull[2], tempty[2], sfull[SF], sempty[SF], drain
   static constexpr uint32_t n_bars = 2 * kStages + 4 + 2 * kSfSmemSlots + 1;
   static constexpr uint32_t misc = align_up(bars + 8 * n_bars, 16);   // tmem slot, abort flag
-  static constexpr uint32_t end = misc + 16;
+  static constexpr uint32_t sched = misc + 16;                        // grouped: int[E + 1]
+  static constexpr uint32_t end = sched + (GROUPED ? 4 * (kMaxGroups + 1) : 0);
   static constexpr uint32_t smem_bytes = end + 1024;
   static_assert(kAccCols + kSfTmemSlots * kSfSlotCols <= static_cast<int>(kTmemCols), "TMEM budget");
   static_assert((kN + 31) / 32 <= 8, "B scales fit two copy blocks");
@@ -114,11 +116,12 @@ __device__ __forceinline__ uint32_t ue8m0_of(float s, bool& bad) {
   return 127;
 }
 
-template <bool ROW_B, bool OUT_BF16>
-__global__ void __launch_bounds__(Ue8m0Cfg::kThreads, 1)
+template <bool ROW_B, bool OUT_BF16, bool GROUPED>
+__global__ void __launch_bounds__(Ue8m0Cfg<GROUPED>::kThreads, 1)
     gemm_fp8_ue8m0_kernel(const __grid_constant__ CUtensorMap tmA,
                           const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
-  using Cfg = Ue8m0Cfg;
+  using Cfg = Ue8m0Cfg<GROUPED>;
+  static_assert(!(GROUPED && ROW_B), "grouped GEMMs take 128x128 weight-block scales");
   constexpr int S = Cfg::kStages;
   constexpr int SF = Cfg::kSfSmemSlots;
   constexpr int TS = Cfg::kSfTmemSlots;
@@ -166,20 +169,36 @@ __global__ void __launch_bounds__(Ue8m0Cfg::kThreads, 1)
     tmem_alloc<1>(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish<1>();
   }
-  const int mt_total = static_cast<int>((p.M + Cfg::kTileM - 1) / Cfg::kTileM);
   const int nt_total = static_cast<int>((p.N + kN - 1) / kN);
-  const int num_tiles = mt_total * nt_total;
+  int* sched = reinterpret_cast<int*>(smem + Cfg::sched);
+  int mt_total = 0, num_tiles = 0;
+  if (!GROUPED) {
+    mt_total = static_cast<int>((p.M + Cfg::kTileM - 1) / Cfg::kTileM);
+    num_tiles = mt_total * nt_total;
+  } else {
+    // per-expert tile counts, then an exclusive prefix (E is small)
+    for (int e = threadIdx.x; e < p.num_experts; e += blockDim.x) {
+      int64_t rb, re;
+      expert_rows(p, e, rb, re);
+      const int64_t rows = re - rb;
+      sched[e + 1] = rows > 0 ? static_cast<int>((rows + Cfg::kTileM - 1) / Cfg::kTileM) * nt_total : 0;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      sched[0] = 0;
+      for (int e = 1; e <= p.num_experts; ++e) sched[e] += sched[e - 1];
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // Tiles of this CTA: blockIdx.x, + gridDim.x, ...; m-fastest so that the CTAs of a
-  // wave share B tiles.
+  if (GROUPED) num_tiles = sched[p.num_experts];
+  // Tiles of this CTA: blockIdx.x, + gridDim.x, ...; dense: m-fastest so that the CTAs
+  // of a wave share B tiles; grouped: expert by expert, n-fastest inside an expert.
   const int n_tiles = blockIdx.x < num_tiles ? (num_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
-  auto tile_of = [&](int i, int64_t& row0, int64_t& col0) {
-    const int t = blockIdx.x + i * gridDim.x;
-    row0 = static_cast<int64_t>(t % mt_total) * Cfg::kTileM;
-    col0 = static_cast<int64_t>(t / mt_total) * kN;
+  auto tile_of = [&](int i) -> Tile {
+    return decode_tile<GROUPED, Cfg::kTileM, kN>(blockIdx.x + i * gridDim.x, p, mt_total, nt_total, sched);
   };
 
   if (warp == 0) {
@@ -188,8 +207,7 @@ __global__ void __launch_bounds__(Ue8m0Cfg::kThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int i = 0; ok && i < n_tiles; ++i) {
-        int64_t row0, col0;
-        tile_of(i, row0, col0);
+        const Tile tl = tile_of(i);
         for (int g = 0; g < G; ++g, ++it) {
           const int s = it % S;
           if (!mbar_wait(empty_bar(s), ((it / S) & 1u) ^ 1u, kSiteProducer, abort_flag)) {
@@ -198,9 +216,9 @@ __global__ void __launch_bounds__(Ue8m0Cfg::kThreads, 1)
           }
           mbar_arrive_expect_tx(full_bar(s), Cfg::kStageTx);
           tma_load_2d(sbase + Cfg::a + s * Cfg::kABytes, &tmA, full_bar(s), g * kBK,
-                      static_cast<int32_t>(row0));
+                      static_cast<int32_t>(tl.row0));
           tma_load_2d(sbase + Cfg::b + s * Cfg::kBBytes, &tmB, full_bar(s), g * kBK,
-                      static_cast<int32_t>(col0));
+                      static_cast<int32_t>(tl.brow0));
         }
       }
       // every issued load lands before the CTA can exit (bounded; loads end on their own)
@@ -279,21 +297,20 @@ __global__ void __launch_bounds__(Ue8m0Cfg::kThreads, 1)
 #pragma unroll
       for (int j = 0; j < kRawB; ++j) raw.b[j] = 1.0f;
       if (i >= n_tiles) return;
-      int64_t row0, col0;
-      tile_of(i, row0, col0);
+      const Tile tl = tile_of(i);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int64_t m = row0 + 32 * j + lane;
+        const int64_t m = tl.row0 + 32 * j + lane;
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
           const int g = 4 * k + b;
-          if (g < G && m < p.M) raw.a[4 * j + b] = __ldg(p.sA + static_cast<int64_t>(g) * p.ld_sa + m);
+          if (g < G && m < tl.row_end) raw.a[4 * j + b] = __ldg(p.sA + static_cast<int64_t>(g) * p.ld_sa + m);
         }
       }
       if (ROW_B) {
 #pragma unroll
         for (int j = 0; j < 7; ++j) {
-          const int64_t n = col0 + 32 * j + lane;
+          const int64_t n = tl.col0 + 32 * j + lane;
 #pragma unroll
           for (int b = 0; b < 4; ++b) {
             const int g = 4 * k + b;
@@ -301,16 +318,16 @@ __global__ void __launch_bounds__(Ue8m0Cfg::kThreads, 1)
           }
         }
       } else {
-        const int64_t nb = col0 / 128 + (lane >> 2);
+        const int64_t nb = tl.col0 / 128 + (lane >> 2);
         const int g = 4 * k + (lane & 3);
-        if (lane < 12 && g < G && nb * 128 < p.N) raw.b[0] = __ldg(p.sB + nb * G + g);
+        if (lane < 12 && g < G && nb * 128 < p.N)
+          raw.b[0] = __ldg(p.sB + (static_cast<int64_t>(tl.expert) * (p.N / 128) + nb) * G + g);
       }
     };
     // Packs the slot into its shared-memory blocks once the MMA thread has copied the
     // ring slot's previous contents.  Returns false (warp-uniform) on abort or timeout.
     auto emit = [&](int i, int64_t sc, const Raw& raw) -> bool {
-      int64_t row0, col0;
-      tile_of(i, row0, col0);
+      const Tile tl = tile_of(i);
       uint32_t wa[4], wb[8];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -334,10 +351,10 @@ __global__ void __launch_bounds__(Ue8m0Cfg::kThreads, 1)
 #pragma unroll
           for (int b = 0; b < 4; ++b) w[jb] |= __shfl_sync(0xFFFFFFFFu, byte, 4 * jb + b) << (8 * b);
         }
-        const int nb0 = static_cast<int>(col0 / 128);
+        const int nb0 = static_cast<int>(tl.col0 / 128);
 #pragma unroll
         for (int j = 0; j < 7; ++j) {
-          const int jb = static_cast<int>((col0 + 32 * j) / 128) - nb0;
+          const int jb = static_cast<int>((tl.col0 + 32 * j) / 128) - nb0;
           wb[j] = jb == 0 ? w[0] : (jb == 1 ? w[1] : w[2]);
         }
       }
@@ -376,24 +393,23 @@ __global__ void __launch_bounds__(Ue8m0Cfg::kThreads, 1)
     const int set = ew >> 2;
     bool ok = true;
     for (int i = 0; i < n_tiles; ++i) {
-      int64_t row0, col0;
-      tile_of(i, row0, col0);
+      const Tile tl = tile_of(i);
       const uint32_t buf = i & 1;
       // warp-uniform outcome: the TMEM loads below are whole-warp instructions
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(tfull_bar(buf), (i >> 1) & 1u, kSiteEpilogue, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      const int64_t m = row0 + 32 * q + lane;
+      const int64_t m = tl.row0 + 32 * q + lane;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + buf * kN +
                              set * Cfg::kSetCols;
-      const int64_t n_set = col0 + set * Cfg::kSetCols;
+      const int64_t n_set = tl.col0 + set * Cfg::kSetCols;
 #pragma unroll 1
       for (int c = 0; c < Cfg::kSetCols; c += 16) {
         uint32_t r[16];
         tmem_ld_16cols(taddr + c, r);
         tmem_ld_wait();
         const int64_t n0 = n_set + c;
-        if (m < p.M && n0 < p.N) {                       // N % 16 == 0: whole chunks
+        if (m < tl.row_end && n0 < p.N) {                // N % 16 == 0: whole chunks
           if (OUT_BF16) {
             uint32_t h[8];
 #pragma unroll

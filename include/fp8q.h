@@ -173,6 +173,18 @@ int fp8_gemm_blockscaled_ue8m0(const uint8_t* A, const float* sA, int64_t ld_sa,
                                int64_t lda, int64_t ldb, int64_t ldc, void* stream);
 
 /*
+ * fp8_gemm_grouped for power-of-two scales, scaled inside the tensor core as in
+ * fp8_gemm_blockscaled_ue8m0 (one expert's rows of A against W[e] per tile, tiles of
+ * 128 x 224).  Same arguments, layouts, requirements and host-side errors as
+ * fp8_gemm_grouped; every scale it reads (sA for rows inside the experts, sW) must be a
+ * power of two in [2^-127, 2^127], otherwise (8 << 8) | FP8Q_ERR_SCALE is recorded as for
+ * fp8_gemm_blockscaled_ue8m0.
+ */
+int fp8_gemm_grouped_ue8m0(const uint8_t* A, const float* sA, int64_t ld_sa, const uint8_t* W,
+                           const float* sW, void* C, int out_dtype, const int32_t* m_offsets,
+                           int num_groups, int64_t max_sum_M, int64_t N, int64_t K, void* stream);
+
+/*
  * Bytes of device workspace that fp8_gemm_blockscaled_ws can use for an M x N x K problem
  * on the current device (0 when splitting the last wave would not help).  *bytes is set
  * on success; K % 128 and N % 128 must be 0.

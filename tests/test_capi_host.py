@@ -123,8 +123,9 @@ def test_gemm_validation(L, entry):
     assert call(ldc=260, out=0) == 3           # 520 B row pitch is not a multiple of 16
 
 
-def test_grouped_validation(L):
-    f = L.fp8_gemm_grouped
+@pytest.mark.parametrize("entry", ["fp8_gemm_grouped", "fp8_gemm_grouped_ue8m0"])
+def test_grouped_validation(L, entry):
+    f = getattr(L, entry)
     assert f(P16, P16, 64, P16, P16, P16, 0, P16, 0, 64, 256, 256, NULL) == 4      # no groups
     assert f(P16, P16, 64, P16, P16, P16, 0, P16, 2000, 64, 256, 256, NULL) == 4   # too many
     assert f(P16, P16, 64, P16, P16, P16, 0, P16, 4, 0, 256, 256, NULL) == 0       # empty

@@ -168,7 +168,7 @@ def test_wgrad_full_size_sampled_rows(fq):
 # ------------------------------------------------------------------------------------ grouped
 
 def _grouped_case(fq, counts, N, K, pow2_a, out_fp32, a_std=1.0, b_std=0.006, rows=None,
-                  seed=0, bits=None, name="grouped", alloc_rows=1):
+                  seed=0, bits=None, name="grouped", alloc_rows=1, pow2_w=False, ue8m0=False):
     import torch
     counts = np.asarray(counts, dtype=np.int64)
     E = counts.size
@@ -181,10 +181,11 @@ def _grouped_case(fq, counts, N, K, pow2_a, out_fp32, a_std=1.0, b_std=0.006, ro
     else:
         a_bits, w_bits = bits
     qa, sa = fq.quant_act_1x128(to_dev_bf16(a_bits), pow2_a)
-    qw, sw = fq.quant_weight_128x128(to_dev_bf16(w_bits), False)
+    qw, sw = fq.quant_weight_128x128(to_dev_bf16(w_bits), pow2_w)
     out_dtype = torch.float32 if out_fp32 else torch.bfloat16
     C = torch.full((max(M, alloc_rows), N), float("nan"), dtype=out_dtype, device="cuda")
-    fq.gemm_grouped(qa, sa, qw, sw, to_dev(off), out_dtype=out_dtype, out=C)
+    gemm = fq.gemm_grouped_ue8m0 if ue8m0 else fq.gemm_grouped
+    gemm(qa, sa, qw, sw, to_dev(off), out_dtype=out_dtype, out=C)
     torch.cuda.synchronize()
     assert fq.device_error() == 0
     assert torch.isnan(C[M:]).all(), "rows past the last offset are not written"
@@ -197,7 +198,7 @@ def _grouped_case(fq, counts, N, K, pow2_a, out_fp32, a_std=1.0, b_std=0.006, ro
     expert = np.searchsorted(off, rows, side="right") - 1
     qw_h, sw_h = host(qw), host(sw)
     for e in np.unique(expert):
-        q_ref, s_ref = oracle.quant_weight_128x128(w_bits[e], False)
+        q_ref, s_ref = oracle.quant_weight_128x128(w_bits[e], pow2_w)
         assert_bytes_equal(f"{name}.qw[{e}]", qw_h[e], q_ref)
         assert_bytes_equal(f"{name}.sw[{e}]", sw_h[e], s_ref)
     # oracle over the sampled rows: sA columns re-indexed to the sampled rows
@@ -205,9 +206,9 @@ def _grouped_case(fq, counts, N, K, pow2_a, out_fp32, a_std=1.0, b_std=0.006, ro
     qa_full[rows] = qa_ref
     sa_full = np.zeros((K // 128, M), np.float32)
     sa_full[:, rows] = sa_ref
-    qw_ref = np.stack([oracle.quant_weight_128x128(w_bits[e], False)[0] if e in expert else
+    qw_ref = np.stack([oracle.quant_weight_128x128(w_bits[e], pow2_w)[0] if e in expert else
                        np.zeros((N, K), np.uint8) for e in range(E)])
-    sw_ref = np.stack([oracle.quant_weight_128x128(w_bits[e], False)[1] if e in expert else
+    sw_ref = np.stack([oracle.quant_weight_128x128(w_bits[e], pow2_w)[1] if e in expert else
                        np.ones((N // 128, K // 128), np.float32) for e in range(E)])
     C_ref, T = oracle.gemm_grouped_ref(qa_full, sa_full, qw_ref, sw_ref, off, rows=rows)
     assert_gemm_close(name, host(C)[rows], C_ref, T, bf16=not out_fp32)
@@ -389,3 +390,49 @@ def test_ue8m0_rejects_scales_that_are_not_powers_of_two(fq):
     fq.gemm_blockscaled_ue8m0(qa2, sa2, qb2, sb2, out_dtype=torch.float32)
     torch.cuda.synchronize()
     assert fq.device_error() == 0
+
+
+# ------------------------------------------- grouped, power-of-two scales in the MMA
+
+@pytest.mark.parametrize("out_fp32", [True, False])
+def test_grouped_ue8m0_ragged_with_empty_groups(fq, out_fp32):
+    """Ragged experts (some empty), N = 384 (a full and a ragged 224-column tile), K = 640
+    (a partial scale slot), slack rows in A; power-of-two scales on both operands."""
+    _grouped_case(fq, [0, 5, 300, 1, 0, 77, 600, 0], 384, 640, True, out_fp32, seed=6,
+                  alloc_rows=1100, pow2_w=True, ue8m0=True, name="grouped ue8m0")
+
+
+def test_grouped_ue8m0_decode_full_size(fq):
+    """The decode workload with power-of-two weight scales: 64 experts, M_e ~ U{1..256},
+    W [7168, 2048]; every 9th row compared."""
+    w = workloads.decode()
+    rows = np.arange(0, w.M, 9)
+    _grouped_case(fq, w.counts, w.N, w.K, True, False, rows=rows, bits=(w.gen_a(), w.gen_b()),
+                  pow2_w=True, ue8m0=True, name="decode ue8m0")
+
+
+def test_grouped_ue8m0_prefill_sampled(fq):
+    """32 experts, Zipf routing (sum M ~ 87K), W [4096, 7168], power-of-two scales; sampled
+    rows of 4 experts."""
+    w = workloads.prefill()
+    off = w.offsets
+    rng = np.random.default_rng(8)
+    rows = []
+    for e in (0, 3, 17, 31):
+        lo, hi = int(off[e]), int(off[e + 1])
+        rows += list(rng.choice(np.arange(lo, hi), 10, replace=False)) + [lo, hi - 1]
+    _grouped_case(fq, w.counts, w.N, w.K, True, False, rows=np.array(sorted(set(rows))),
+                  bits=(w.gen_a(), w.gen_b()), pow2_w=True, ue8m0=True, name="prefill ue8m0")
+
+
+def test_grouped_ue8m0_rejects_fp32_weight_scales(fq):
+    import torch
+    rng = np.random.default_rng(9)
+    a = workloads.normal_bf16(rng, (200, 256), 1.0)
+    w = workloads.normal_bf16(rng, (2, 256, 256), 0.02)
+    qa, sa = fq.quant_act_1x128(to_dev_bf16(a), True)
+    qw, sw = fq.quant_weight_128x128(to_dev_bf16(w), False)       # FP32 scales
+    off = to_dev(workloads.offsets_from_counts(np.array([120, 80])))
+    fq.gemm_grouped_ue8m0(qa, sa, qw, sw, off)
+    torch.cuda.synchronize()
+    assert fq.device_error() == (8 << 8) | 7
