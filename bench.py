@@ -521,15 +521,17 @@ def profile_case(args, name: str, launches: int = 3):
             raise RuntimeError("device error word set")
         print(json.dumps({"profile_case": "quant_act_dual_16384x7168", "launches": launches}), flush=True)
         return
-    w = workloads.ALL[name]()
+    pow2_grouped = name == "decode_pow2"   # decode with power-of-two weight scales too
+    w = workloads.ALL["decode" if pow2_grouped else name]()
     if w.experts:
         off = torch.from_numpy(w.offsets).cuda()
         A = _dev_normal((w.M, w.K), w.a_std, 7001)
         W = _dev_normal((w.experts, w.N, w.K), w.b_std, 7002)
-        qA, sA = fq.quant_act_1x128(A, w.pow2_a)
-        qW, sW = fq.quant_weight_128x128(W, w.pow2_b)
+        qA, sA = fq.quant_act_1x128(A, w.pow2_a or pow2_grouped)
+        qW, sW = fq.quant_weight_128x128(W, w.pow2_b or pow2_grouped)
         C = torch.empty((w.M, w.N), dtype=torch.bfloat16, device="cuda")
-        run = lambda: fq.gemm_grouped(qA, sA, qW, sW, off, out=C)
+        gemm = fq.gemm_grouped_ue8m0 if pow2_grouped else fq.gemm_grouped
+        run = lambda: gemm(qA, sA, qW, sW, off, out=C)
     else:
         A = _dev_normal((w.M, w.K), w.a_std, 7001)
         B = _dev_normal((w.N, w.K), w.b_std, 7002)
@@ -661,7 +663,8 @@ def main():
     ap.add_argument("--no-check", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' timings")
     ap.add_argument("--no-study", action="store_true", help="skip the accumulation study")
-    ap.add_argument("--profile-case", choices=["tiny", "dense", "prefill", "decode", "wgrad", "dual"],
+    ap.add_argument("--profile-case",
+                    choices=["tiny", "dense", "prefill", "decode", "decode_pow2", "wgrad", "dual"],
                     help="only run a few GEMM launches of one workload (for ncu) and exit")
     args = ap.parse_args()
 
