@@ -402,6 +402,12 @@ def test_grouped_ue8m0_ragged_with_empty_groups(fq, out_fp32):
                   alloc_rows=1100, pow2_w=True, ue8m0=True, name="grouped ue8m0")
 
 
+def test_grouped_ue8m0_all_empty(fq):
+    """Every expert empty: no tiles, the call is a clean no-op (C untouched)."""
+    _grouped_case(fq, [0, 0, 0], 256, 256, True, True, seed=10, pow2_w=True, ue8m0=True,
+                  name="grouped ue8m0 empty")
+
+
 def test_grouped_ue8m0_decode_full_size(fq):
     """The decode workload with power-of-two weight scales: 64 experts, M_e ~ U{1..256},
     W [7168, 2048]; every 9th row compared."""
