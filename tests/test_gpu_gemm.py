@@ -408,6 +408,16 @@ def test_grouped_ue8m0_all_empty(fq):
                   name="grouped ue8m0 empty")
 
 
+@pytest.mark.parametrize("ue8m0", [False, True])
+def test_grouped_maximum_expert_count(fq, ue8m0):
+    """1024 experts (the largest table the kernels hold), all but the first, a middle and
+    the last one empty: the tile table's ends and its binary search."""
+    counts = np.zeros(1024, np.int64)
+    counts[0], counts[511], counts[1023] = 5, 130, 7
+    _grouped_case(fq, counts, 128, 256, True, True, seed=11, pow2_w=ue8m0, ue8m0=ue8m0,
+                  name=f"1024 experts ue8m0={ue8m0}")
+
+
 def test_grouped_ue8m0_decode_full_size(fq):
     """The decode workload with power-of-two weight scales: 64 experts, M_e ~ U{1..256},
     W [7168, 2048]; every 9th row compared."""
