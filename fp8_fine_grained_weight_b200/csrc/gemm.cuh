@@ -27,15 +27,17 @@
 //               128*((w-4)/4)..; per group: tcgen05.ld -> acc += P * scale in FP32
 //               registers; at tile end: convert and store C.
 //
-// PAIR = true: two CTAs of a cluster share a 256 x 256 output tile with
-// tcgen05 cta_group::2.  Each CTA loads its own 128 rows of A and 128 of the 256 rows
-// of B (32 KB per stage instead of 48 KB, so 6 stages fit), the even CTA issues the
-// M = 256 MMAs and its commits arrive on both CTAs' barriers; each CTA's TMEM holds
-// its 128 rows x 256 columns and its own epilogue promotes them; the odd CTA frees an
-// accumulator buffer with a remote arrive on the even CTA's barrier.  No TMA multicast:
-// every CTA loads its own operands.
+// PAIR = true: two CTAs of a cluster share a 256 x 128 output tile with tcgen05
+// cta_group::2.  Each CTA loads its own 128 rows of A and 64 of the 128 rows of B (24 KB
+// per stage, 8 stages), the even CTA issues the M = 256 MMAs and its commits arrive on
+// both CTAs' barriers; each CTA's TMEM holds four 128-column accumulator buffers for its
+// 128 rows and its own epilogue promotes them; the odd CTA frees a buffer with a remote
+// arrive on the even CTA's barrier.  No TMA multicast: every CTA loads its own operands.
+// It passes the parity tests but measures slower than the single-CTA tile (its groups
+// are half as large, so the per-group hand-off is paid twice as often); the launcher
+// does not instantiate it.
 // PAIR = false (used by the promoted GEMMs): one CTA per 128 x 256 tile, B tile of 256
-// rows, 4 stages; every accumulator release is a local barrier arrive.
+// rows, 4 stages, two 256-column accumulator buffers; every release is a local arrive.
 //
 // Registers: the launch gives 168 per thread (3 warps per SM sub-partition).  The
 // first warpgroup gives registers back (setmaxnreg 56) and the two epilogue

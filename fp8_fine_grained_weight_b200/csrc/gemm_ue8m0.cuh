@@ -18,9 +18,13 @@
 // with scale 1.
 //
 // Tiles of 128 x 224 (224 divides 7168; two 224-column FP32 accumulators and the scale
-// region fill the 512 TMEM columns), persistent CTAs, 12 warps:
+// region fill the 512 TMEM columns), persistent CTAs, 12 warps.  GROUPED: the MoE form of
+// fp8_gemm_grouped -- tiles come from a per-expert table built from m_offsets on the
+// device (n fastest inside an expert), A rows past an expert's end are masked, B rows
+// come from the stacked expert weights with that expert's block scales, and the ring has
+// 4 stages to leave room for the table.
 //   warp 0       TMA producer: A [128 x 128 B] and B [224 x 128 B] per K-group into a
-//                5-stage ring (128-byte swizzle).
+//                5-stage ring (4 when grouped; 128-byte swizzle).
 //   warp 1       TMEM owner and MMA issuer.  Per slot of four groups it copies the slot's
 //                scale words from shared memory into TMEM (tcgen05.cp 32x128b.warpx4: a
 //                32-row x 16-byte block into 4 columns of every 32-lane sub-partition),
