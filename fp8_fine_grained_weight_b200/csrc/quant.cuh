@@ -216,18 +216,21 @@ __global__ void __launch_bounds__(256) quant_act_1x128_kernel(const uint16_t* __
 //
 // Grid (M/128, K/128), 256 threads, one 128x128 tile of X per block:
 //  rows:    as quant_act_1x128_kernel (teams of 4 lanes per row, 16 rows per warp), all
-//           eight 16-byte loads of a thread issued before any arithmetic; the tile is
-//           kept in shared memory (row pitch 256 bytes);
-//  columns: thread t owns the column pair 2 (t % 64), +1 and rows 32 (t / 64) .. + 31 of
-//           the tile (32-bit shared loads); the four quarters' amax meet in shared memory;
-//           the codes are staged transposed in the tile's space once every thread has
-//           read it (row pitch kDualPitch bytes) and written as 128-byte column segments.
+//           eight 16-byte loads of a thread in flight before any arithmetic; the tile is
+//           kept in shared memory with a 320-byte row pitch (the two rows a quarter-warp
+//           stores land 16 banks apart);
+//  columns: thread t owns the column pair 2 (t % 64), +1 and rows 32 (t / 64) .. + 31,
+//           read once into registers (32-bit shared loads); the four quarters' amax meet
+//           in shared memory; the codes are staged transposed in the tile's space once
+//           every thread has read it (row pitch kDualPitch bytes) and written as 128-byte
+//           column segments.  4 CTAs per SM (the 32 column words live in registers).
 constexpr int kDualPitch = 144;                     // 128 codes + 16
-constexpr int kDualSmem = 128 * 256 + 4 * 64 * 4;  // tile (reused for the codes) + amax parts
-static_assert(128 * kDualPitch <= 128 * 256, "codes fit in the tile's space");
+constexpr int kDualRowPitch = 320;                 // bf16 tile rows: alternate rows 16 banks apart
+constexpr int kDualSmem = 128 * kDualRowPitch + 4 * 64 * 4;   // tile (reused for the codes) + amax parts
+static_assert(128 * kDualPitch <= 128 * kDualRowPitch, "codes fit in the tile's space");
 
 template <bool POW2>
-__global__ void __launch_bounds__(256, 5) quant_act_dual_kernel(const uint16_t* __restrict__ x,
+__global__ void __launch_bounds__(256, 4) quant_act_dual_kernel(const uint16_t* __restrict__ x,
                                                              int64_t ldx, uint8_t* __restrict__ q,
                                                              int64_t ldq, float* __restrict__ s,
                                                              int64_t lds, uint8_t* __restrict__ qt,
@@ -235,7 +238,7 @@ __global__ void __launch_bounds__(256, 5) quant_act_dual_kernel(const uint16_t* 
                                                              int64_t ldst) {
   extern __shared__ __align__(16) uint8_t dual_smem[];
   uint8_t* tile = dual_smem;                               // bf16 [128][128], then E4M3 codes
-  uint32_t* part = reinterpret_cast<uint32_t*>(dual_smem + 128 * 256);   // [4][64] amax pairs
+  uint32_t* part = reinterpret_cast<uint32_t*>(dual_smem + 128 * kDualRowPitch);   // [4][64] amax pairs
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int l4 = lane & 3;
   const int64_t m0 = static_cast<int64_t>(blockIdx.x) * 128;
@@ -256,7 +259,7 @@ __global__ void __launch_bounds__(256, 5) quant_act_dual_kernel(const uint16_t* 
     const int r = warp * 16 + pass * 8 + (lane >> 2);      // row inside the tile
     const int64_t m = m0 + r;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(tile + r * 256 + (l4 + 4 * j) * 16) = v[pass][j];
+    for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(tile + r * kDualRowPitch + (l4 + 4 * j) * 16) = v[pass][j];
     float a = amax_vectors(v[pass]);
     a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
     a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
@@ -273,10 +276,14 @@ __global__ void __launch_bounds__(256, 5) quant_act_dual_kernel(const uint16_t* 
 
   // ---- columns 2p, 2p+1 over rows 32h .. 32h + 31
   const int p = threadIdx.x & 63, h = threadIdx.x >> 6;
-  const uint32_t* words = reinterpret_cast<const uint32_t*>(tile) + p;   // row r: words[64 r]
+  const uint32_t* words = reinterpret_cast<const uint32_t*>(tile) + p;   // row r: words[80 r]
+  uint32_t wv[32];
   uint32_t mx = 0;
-#pragma unroll 8
-  for (int r = 0; r < 32; ++r) mx = __vmaxu2(mx, words[(32 * h + r) * 64] & 0x7FFF7FFFu);
+#pragma unroll
+  for (int r = 0; r < 32; ++r) {
+    wv[r] = words[(32 * h + r) * (kDualRowPitch / 4)];
+    mx = __vmaxu2(mx, wv[r] & 0x7FFF7FFFu);
+  }
   part[h * 64 + p] = mx;
   __syncthreads();
   const uint32_t mall = __vmaxu2(__vmaxu2(part[p], part[64 + p]), __vmaxu2(part[128 + p], part[192 + p]));
@@ -289,9 +296,8 @@ __global__ void __launch_bounds__(256, 5) quant_act_dual_kernel(const uint16_t* 
   auto codes_with = [&](auto f_lo, auto f_hi) {
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
-      const int r = 32 * h + 4 * w;
-      const uint32_t w0 = words[r * 64], w1 = words[(r + 1) * 64];
-      const uint32_t w2 = words[(r + 2) * 64], w3 = words[(r + 3) * 64];
+      const uint32_t w0 = wv[4 * w], w1 = wv[4 * w + 1];
+      const uint32_t w2 = wv[4 * w + 2], w3 = wv[4 * w + 3];
       c_lo[w] = cvt_e4m3x2(f_lo(bf16lo(w0)), f_lo(bf16lo(w1))) |
                 (cvt_e4m3x2(f_lo(bf16lo(w2)), f_lo(bf16lo(w3))) << 16);
       c_hi[w] = cvt_e4m3x2(f_hi(bf16hi(w0)), f_hi(bf16hi(w1))) |
