@@ -564,10 +564,11 @@ def gemm_path(args, w) -> str:
 
 
 def kernel_rev() -> str:
-    """Short hash of the kernel sources, to tie stored ncu counters to the code they measured."""
+    """Short hash of the GEMM sources (the kernels and their launch code), to tie stored
+    ncu counters of a GEMM to the code they measured."""
     import hashlib
     h = hashlib.sha1()
-    for f in ("ptx.cuh", "quant.cuh", "gemm.cuh", "gemm_ue8m0.cuh", "fp8q.cu"):
+    for f in ("ptx.cuh", "gemm.cuh", "gemm_ue8m0.cuh", "fp8q.cu"):
         h.update(open(os.path.join(ROOT, "fp8_fine_grained_weight_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:12]
 
