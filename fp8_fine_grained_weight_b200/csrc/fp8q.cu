@@ -341,15 +341,16 @@ int fp8q_quant_act_1x128(const void* x, int64_t M, int64_t K, int64_t ldx, uint8
   if (ldx % 8 != 0 || ldq % 8 != 0 || !aligned(x, 16) || !aligned(q, 8) || !aligned(scales, 4))
     return FP8Q_ERR_ALIGN;
   const int64_t G = K / 128;
-  if (G > 65535) return FP8Q_ERR_SHAPE;
-  dim3 grid(static_cast<unsigned>((M + fp8q::kActRowsPerBlock - 1) / fp8q::kActRowsPerBlock),
-            static_cast<unsigned>(G));
+  const int64_t row_blocks = M / fp8q::kActRowsPerBlock + (M % fp8q::kActRowsPerBlock != 0);
+  if (row_blocks > 0x7FFFFFFF / G) return FP8Q_ERR_SHAPE;   // one-dimensional grid
+  const unsigned grid = static_cast<unsigned>(row_blocks * G);
   auto st = static_cast<cudaStream_t>(stream);
   const auto* xs = static_cast<const uint16_t*>(x);
+  const auto g32 = static_cast<uint32_t>(G);
   if (pow2_scale)
-    fp8q::quant_act_1x128_kernel<true><<<grid, 256, 0, st>>>(xs, M, ldx, q, ldq, scales, ld_scale);
+    fp8q::quant_act_1x128_kernel<true><<<grid, 256, 0, st>>>(xs, M, ldx, q, ldq, scales, ld_scale, g32);
   else
-    fp8q::quant_act_1x128_kernel<false><<<grid, 256, 0, st>>>(xs, M, ldx, q, ldq, scales, ld_scale);
+    fp8q::quant_act_1x128_kernel<false><<<grid, 256, 0, st>>>(xs, M, ldx, q, ldq, scales, ld_scale, g32);
   return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
@@ -364,7 +365,7 @@ int fp8q_quant_act_dual(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
   if (ldx % 8 != 0 || ldq % 8 != 0 || ldqt % 16 != 0 || !aligned(x, 16) || !aligned(q, 8) ||
       !aligned(qt, 16) || !aligned(s, 4) || !aligned(st, 4))
     return FP8Q_ERR_ALIGN;
-  if (K / 128 > 65535 || M / 128 > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
+  if (M / 128 > 0x7FFFFFFF / (K / 128)) return FP8Q_ERR_SHAPE;   // one-dimensional grid
   static std::atomic<unsigned long long> ready{0};   // per-device bit: attributes set
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8Q_ERR_CUDA;
@@ -376,15 +377,16 @@ int fp8q_quant_act_dual(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
       return FP8Q_ERR_CUDA;
     ready.fetch_or(1ull << dev, std::memory_order_acq_rel);
   }
-  dim3 grid(static_cast<unsigned>(M / 128), static_cast<unsigned>(K / 128));
+  const unsigned grid = static_cast<unsigned>((M / 128) * (K / 128));
+  const auto g32 = static_cast<uint32_t>(K / 128);
   auto stm = static_cast<cudaStream_t>(stream);
   const auto* xs = static_cast<const uint16_t*>(x);
   if (pow2_scale)
     fp8q::quant_act_dual_kernel<true><<<grid, 256, fp8q::kDualSmem, stm>>>(xs, ldx, q, ldq, s, ld_s, qt,
-                                                                           ldqt, st, ld_st);
+                                                                           ldqt, st, ld_st, g32);
   else
     fp8q::quant_act_dual_kernel<false><<<grid, 256, fp8q::kDualSmem, stm>>>(xs, ldx, q, ldq, s, ld_s, qt,
-                                                                            ldqt, st, ld_st);
+                                                                            ldqt, st, ld_st, g32);
   return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 

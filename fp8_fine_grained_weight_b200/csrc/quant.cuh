@@ -164,23 +164,27 @@ __device__ __forceinline__ void stg_u2(void* p, uint2 v) {
 
 // ---------------------------------------------------------------- 1x128 activation tiles
 //
-// Grid (ceil(M / 64), G), 256 threads.  A team of 4 lanes owns one row's 128-element
-// group: lane l of the team holds the 16-byte chunks l, l+4, l+8, l+12 (so each load
-// instruction reads 64 contiguous bytes per team), all four loads in flight before any
-// arithmetic.  The amax needs two xor-shuffles inside the team; the scale and its
-// reciprocal are computed once per lane for 32 elements.  A warp covers 8 consecutive
-// rows of one group, so lane 0 of each team writes 8 consecutive scale words.
+// One 256-thread block per (64-row block, 128-column group).  A team of 4 lanes owns one
+// row's 128-element group: lane l of the team holds the 16-byte chunks l, l+4, l+8, l+12
+// (so each load instruction reads 64 contiguous bytes per team), all four loads in
+// flight before any arithmetic.  The amax needs two xor-shuffles inside the team; the
+// scale and its reciprocal are computed once per lane for 32 elements.  A warp covers 8
+// consecutive rows of one group, so lane 0 of each team writes 8 consecutive scale words.
+//
+// The grid is one-dimensional with the group index fastest: consecutive blocks read
+// adjacent 256-byte segments of the same 64 rows, which keeps their DRAM accesses in
+// the same pages (on B200 about 9% faster than the row block running fastest, measured
+// on [16384, 7168] with L2 flushed between launches).
 constexpr int kActRowsPerBlock = 64;
 
 template <bool POW2>
-__global__ void __launch_bounds__(256) quant_act_1x128_kernel(const uint16_t* __restrict__ x,
-                                                              int64_t M, int64_t ldx,
-                                                              uint8_t* __restrict__ q, int64_t ldq,
-                                                              float* __restrict__ s, int64_t lds) {
+__device__ __forceinline__ void quant_act_1x128_tile(const uint16_t* __restrict__ x, int64_t M,
+                                                     int64_t ldx, uint8_t* __restrict__ q,
+                                                     int64_t ldq, float* __restrict__ s,
+                                                     int64_t lds, int64_t rb, int64_t g) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int l4 = lane & 3;
-  const int64_t g = blockIdx.y;
-  const int64_t m = static_cast<int64_t>(blockIdx.x) * kActRowsPerBlock + warp * 8 + (lane >> 2);
+  const int64_t m = rb * kActRowsPerBlock + warp * 8 + (lane >> 2);
   const bool valid = m < M;
   const uint16_t* src = x + m * ldx + g * 128 + l4 * 8;
 
@@ -202,6 +206,16 @@ __global__ void __launch_bounds__(256) quant_act_1x128_kernel(const uint16_t* __
   }
 }
 
+// Grid (ceil(M / 64) * G): block b covers group b % G of row block b / G.
+template <bool POW2>
+__global__ void __launch_bounds__(256) quant_act_1x128_kernel(const uint16_t* __restrict__ x,
+                                                              int64_t M, int64_t ldx,
+                                                              uint8_t* __restrict__ q, int64_t ldq,
+                                                              float* __restrict__ s, int64_t lds,
+                                                              uint32_t G) {
+  quant_act_1x128_tile<POW2>(x, M, ldx, q, ldq, s, lds, blockIdx.x / G, blockIdx.x % G);
+}
+
 // ---------------------------------------------------------------- rows and columns in one pass
 //
 // One HBM read of a bf16 activation X [M, K] produces both
@@ -214,7 +228,9 @@ __global__ void __launch_bounds__(256) quant_act_1x128_kernel(const uint16_t* __
 // The Wgrad GEMM consumes the transposed copy; this kernel reads each element once for
 // both copies.
 //
-// Grid (M/128, K/128), 256 threads, one 128x128 tile of X per block:
+// Grid (M/128 * K/128), 256 threads, one 128x128 tile of X per block, the column group
+// running fastest (block b: group b % (K/128) of row tile b / (K/128), as for the 1x128
+// kernel):
 //  rows:    as quant_act_1x128_kernel (teams of 4 lanes per row, 16 rows per warp), all
 //           eight 16-byte loads of a thread in flight before any arithmetic; the tile is
 //           kept in shared memory with a 320-byte row pitch (the two rows a quarter-warp
@@ -230,20 +246,19 @@ constexpr int kDualSmem = 128 * kDualRowPitch + 4 * 64 * 4;   // tile (reused fo
 static_assert(128 * kDualPitch <= 128 * kDualRowPitch, "codes fit in the tile's space");
 
 template <bool POW2>
-__global__ void __launch_bounds__(256, 4) quant_act_dual_kernel(const uint16_t* __restrict__ x,
-                                                             int64_t ldx, uint8_t* __restrict__ q,
-                                                             int64_t ldq, float* __restrict__ s,
-                                                             int64_t lds, uint8_t* __restrict__ qt,
-                                                             int64_t ldqt, float* __restrict__ st,
-                                                             int64_t ldst) {
+__device__ __forceinline__ void quant_act_dual_tile(const uint16_t* __restrict__ x, int64_t ldx,
+                                                    uint8_t* __restrict__ q, int64_t ldq,
+                                                    float* __restrict__ s, int64_t lds,
+                                                    uint8_t* __restrict__ qt, int64_t ldqt,
+                                                    float* __restrict__ st, int64_t ldst,
+                                                    int64_t rb, int64_t g) {
   extern __shared__ __align__(16) uint8_t dual_smem[];
   uint8_t* tile = dual_smem;                               // bf16 [128][128], then E4M3 codes
   uint32_t* part = reinterpret_cast<uint32_t*>(dual_smem + 128 * kDualRowPitch);   // [4][64] amax pairs
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int l4 = lane & 3;
-  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * 128;
-  const int64_t k0 = static_cast<int64_t>(blockIdx.y) * 128;
-  const int64_t g = blockIdx.y;
+  const int64_t m0 = rb * 128;
+  const int64_t k0 = g * 128;
 
   // ---- rows: both passes' loads first
   uint4 v[2][4];
@@ -345,6 +360,16 @@ __global__ void __launch_bounds__(256, 4) quant_act_dual_kernel(const uint16_t* 
     const uint4 val = *reinterpret_cast<const uint4*>(codes + cc * kDualPitch + chunk * 16);
     *reinterpret_cast<uint4*>(qt + (k0 + cc) * ldqt + m0 + chunk * 16) = val;
   }
+}
+
+template <bool POW2>
+__global__ void __launch_bounds__(256, 4) quant_act_dual_kernel(const uint16_t* __restrict__ x,
+                                                             int64_t ldx, uint8_t* __restrict__ q,
+                                                             int64_t ldq, float* __restrict__ s,
+                                                             int64_t lds, uint8_t* __restrict__ qt,
+                                                             int64_t ldqt, float* __restrict__ st,
+                                                             int64_t ldst, uint32_t G) {
+  quant_act_dual_tile<POW2>(x, ldx, q, ldq, s, lds, qt, ldqt, st, ldst, blockIdx.x / G, blockIdx.x % G);
 }
 
 // ---------------------------------------------------------------- transposed weight blocks
