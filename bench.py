@@ -310,6 +310,7 @@ def run_gpu(args, rank, world):
 
     if rank == 0 and not args.no_configs:
         res["configs"] = config_throughput(fq, flush_l2)
+        res["library_fp8_ceiling"] = library_fp8_ceiling(flush_l2)
     if rank == 0 and not args.no_study:
         res["accumulation_study"] = accumulation_study(fq)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -453,6 +454,34 @@ def config_throughput(fq, flush_l2, reps=10):
                          "tflops_3_gemms": round(tf, 1), "frac_of_fp8_peak": round(tf / fp8_peak, 4),
                          "launches": 7}
     return out
+
+
+def library_fp8_ceiling(flush_l2, n: int = 8192, reps: int = 20) -> dict:
+    """The box's FP8 GEMM ceiling as a vendor library reaches it: torch._scaled_mm
+    (cuBLASLt) on [n, n] x [n, n]^T E4M3 operands with one FP32 scale per tensor, bf16 out,
+    L2 flushed before each launch.  Context for the block-scaled kernels' fraction of peak,
+    not one of this library's kernels and not part of the timed step.  A failure is
+    reported in the result, never raised."""
+    try:
+        import torch
+        g = torch.Generator(device="cuda")
+        g.manual_seed(7001)
+        a = torch.randn(n, n, generator=g, device="cuda").to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, generator=g, device="cuda").to(torch.float8_e4m3fn)
+        one = torch.ones((), dtype=torch.float32, device="cuda")
+
+        def mm():
+            return torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+
+        t = _time_ms(mm, reps, flush_l2, warmup=5)
+        del a, b
+        _, bf16_burst, _, _ = peaks()
+        tf = 2.0 * n * n * n / (t * 1e-3) / 1e12
+        return {"call": "torch._scaled_mm (cuBLASLt), E4M3, per-tensor scales, bf16 out",
+                "M": n, "N": n, "K": n, "ms": round(t, 4), "tflops": round(tf, 1),
+                "frac_of_fp8_peak": round(tf / (FP8_PER_BF16 * bf16_burst), 4)}
+    except Exception as e:     # reported, not raised: this leg is context only
+        return {"unavailable": f"{type(e).__name__}: {str(e).splitlines()[0][:200] if str(e) else ''}"}
 
 
 def accumulation_study(fq, rows_sampled=32):

@@ -53,6 +53,18 @@ def test_gemm_path_follows_the_scales():
         bench.gemm_path(SimpleNamespace(gemm="ue8m0"), wgrad)
 
 
+def test_library_ceiling_reports_instead_of_raising():
+    """The cuBLASLt FP8 ceiling leg is context only: without a usable GPU it returns an
+    'unavailable' entry and the bench line is still printed."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present: the leg would measure instead")
+    flushed = []
+    got = bench.library_fp8_ceiling(lambda: flushed.append(1), n=256, reps=1)
+    assert set(got) == {"unavailable"} and got["unavailable"]
+    json.dumps(got)
+
+
 def _run_bench(*args, env=None):
     e = dict(os.environ, **(env or {}))
     return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], cwd=ROOT,
