@@ -71,7 +71,9 @@ typedef enum {
  * q       device, E4M3 bytes [M, K], row stride ldq bytes
  * scales  device, fp32, group-major: [K/128][ld_scale], ld_scale >= M
  * Requires K % 128 == 0, ldx >= K and ldx % 8 == 0, ldq >= K and ldq % 8 == 0,
- * x and q 16- and 8-byte aligned.  Output is bit-exact with the definition above.
+ * x and q 16- and 8-byte aligned, and ceil(M/64) * (K/128) <= 2^31 - 1 (one thread
+ * block per 64 rows x 128 columns); otherwise FP8Q_ERR_SHAPE / FP8Q_ERR_ALIGN before
+ * any launch.  Output is bit-exact with the definition above.
  */
 int fp8q_quant_act_1x128(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
                          int64_t ldq, float* scales, int64_t ld_scale, int pow2_scale, void* stream);
@@ -103,7 +105,9 @@ int fp8q_quant_weight_128x128(const void* w_bf16, int64_t N, int64_t K, int64_t 
  *         the amax of x[128 (m/128) .. +127, k]
  * st      device, fp32 group-major [M/128][ld_st >= K]: st[(m/128) * ld_st + k]
  * Requires M % 128 == 0, K % 128 == 0, ldx % 8 == 0, ldq % 8 == 0, ldqt % 16 == 0,
- * x and qt 16-byte aligned, q 8-byte aligned.  Both outputs are bit-exact with the
+ * x and qt 16-byte aligned, q 8-byte aligned, and (M/128) * (K/128) <= 2^31 - 1 (one
+ * thread block per 128x128 tile); otherwise FP8Q_ERR_SHAPE / FP8Q_ERR_ALIGN before any
+ * launch.  Both outputs are bit-exact with the
  * definition (the qt / st pair equals fp8q_quant_act_1x128 applied to X^T).
  */
 int fp8q_quant_act_dual(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, uint8_t* q,

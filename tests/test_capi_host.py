@@ -67,6 +67,12 @@ def test_quant_act_validation(L):
     assert f(P16, 4, 128, 128, P16, 128, P16, 3, 0, NULL) == 2          # ld_scale < M
     assert f(P_MIS, 4, 128, 128, P16, 128, P16, 4, 0, NULL) == 3        # x misaligned
     assert f(P16, 4, 128, 132, P16, 128, P16, 4, 0, NULL) == 3          # ldx % 8
+    # one block per (64-row block, 128-column group) on a one-dimensional grid of at
+    # most 2^31 - 1 blocks
+    M = 64 << 30
+    assert f(P16, M, 256, 256, P16, 256, P16, M, 0, NULL) == 2         # 2^31 blocks
+    M = 64 << 31
+    assert f(P16, M, 128, 128, P16, 128, P16, M, 0, NULL) == 2
 
 
 def test_quant_dual_validation(L):
@@ -86,6 +92,8 @@ def test_quant_dual_validation(L):
     assert call(ldqt=264) == 3                  # 16-byte row starts of qt
     assert call(qt=P_MIS) == 3
     assert call(x=P_MIS) == 3
+    M = 128 << 30                               # 2^30 row tiles x 2 groups = 2^31 blocks
+    assert call(M=M, ld_s=M, ldqt=M) == 2
 
 
 def test_quant_weight_validation(L):
