@@ -93,9 +93,13 @@ def _stream(t: torch.Tensor) -> int:
     return torch.cuda.current_stream(t.device).cuda_stream
 
 
-def _need(t: torch.Tensor, dtype, name: str, ndim: Optional[int] = None) -> None:
+def _require_cuda(t: torch.Tensor, name: str) -> None:
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA tensor")
+
+
+def _need(t: torch.Tensor, dtype, name: str, ndim: Optional[int] = None) -> None:
+    _require_cuda(t, name)
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if ndim is not None and t.dim() != ndim:
@@ -108,6 +112,30 @@ def _u8(t: torch.Tensor) -> torch.Tensor:
     return t.view(torch.uint8) if t.dtype == torch.float8_e4m3fn else t
 
 
+def _same_device(t: torch.Tensor, device: torch.device, name: str) -> None:
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the other operands on {device}")
+
+
+def _rows(t: torch.Tensor, dtype, name: str, rows: int, cols: int, device: torch.device) -> None:
+    """A 2-D operand the kernels address as [rows, cols] through its row stride: on `device`,
+    contiguous in its last dimension and at least rows x cols (the library sees only a
+    pointer and the stride, so a smaller tensor would be read or written out of bounds)."""
+    _need(t, dtype, name, 2)
+    _same_device(t, device, name)
+    if t.shape[0] < rows or t.shape[1] < cols:
+        raise ValueError(f"{name} must be at least [{rows}, {cols}], got {tuple(t.shape)}")
+
+
+def _dense(t: torch.Tensor, dtype, name: str, shape, device: torch.device) -> None:
+    """An operand the kernels address with an implied row pitch: exactly `shape`, contiguous."""
+    _need(t, dtype, name)
+    _same_device(t, device, name)
+    if tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous tensor of shape {tuple(shape)}, "
+                         f"got {tuple(t.shape)} with strides {t.stride()}")
+
+
 # --------------------------------------------------------------------------------------
 # quantization
 # --------------------------------------------------------------------------------------
@@ -117,14 +145,19 @@ def quant_act_1x128(x: torch.Tensor, pow2: bool = False, ld_scale: Optional[int]
     """1x128 activation tiles: x bf16 [M, K] -> (q uint8 [M, K], s fp32 [K/128, ld_scale])."""
     _need(x, torch.bfloat16, "x", 2)
     M, K = x.shape
-    ld = M if ld_scale is None else int(ld_scale)
     if out is None:
+        ld = M if ld_scale is None else int(ld_scale)
         q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
         s = torch.empty((K // 128 if K % 128 == 0 else 0, ld), dtype=torch.float32, device=x.device)
     else:
         q, s = out
-    _call("fp8q_quant_act_1x128", x.data_ptr(), M, K, x.stride(0), q.data_ptr(), q.stride(0),
-          s.data_ptr(), ld, int(bool(pow2)), _stream(x))
+        _rows(_u8(q), torch.uint8, "q", M, K, x.device)
+        _rows(s, torch.float32, "s", K // 128, M, x.device)
+        ld = s.stride(0)
+        if ld_scale is not None and int(ld_scale) != ld:
+            raise ValueError(f"ld_scale {ld_scale} disagrees with the row stride {ld} of s")
+    _call("fp8q_quant_act_1x128", x.data_ptr(), M, K, x.stride(0), _u8(q).data_ptr(),
+          _u8(q).stride(0), s.data_ptr(), ld, int(bool(pow2)), _stream(x))
     return q, s
 
 
@@ -141,8 +174,13 @@ def quant_act_dual(x: torch.Tensor, pow2: bool = False, out=None):
         st = torch.empty((M // 128, K), dtype=torch.float32, device=x.device)
     else:
         q, s, qt, st = out
-    _call("fp8q_quant_act_dual", x.data_ptr(), M, K, x.stride(0), q.data_ptr(), q.stride(0),
-          s.data_ptr(), s.stride(0), qt.data_ptr(), qt.stride(0), st.data_ptr(), st.stride(0),
+        _rows(_u8(q), torch.uint8, "q", M, K, x.device)
+        _rows(s, torch.float32, "s", K // 128, M, x.device)
+        _rows(_u8(qt), torch.uint8, "qt", K, M, x.device)
+        _rows(st, torch.float32, "st", M // 128, K, x.device)
+    q8, qt8 = _u8(q), _u8(qt)
+    _call("fp8q_quant_act_dual", x.data_ptr(), M, K, x.stride(0), q8.data_ptr(), q8.stride(0),
+          s.data_ptr(), s.stride(0), qt8.data_ptr(), qt8.stride(0), st.data_ptr(), st.stride(0),
           int(bool(pow2)), _stream(x))
     return q, s, qt, st
 
@@ -154,15 +192,16 @@ def transpose_blocks(q: torch.Tensor, s: torch.Tensor, out=None):
     _need(q, torch.uint8, "q", 2)
     _need(s, torch.float32, "s", 2)
     N, K = q.shape
-    if not s.is_contiguous():
-        raise ValueError("s must be contiguous")
+    _dense(s, torch.float32, "s", (N // 128, K // 128), q.device)
     if out is None:
         qt = torch.empty((K, N), dtype=torch.uint8, device=q.device)
         st = torch.empty((K // 128, N // 128), dtype=torch.float32, device=q.device)
     else:
         qt, st = out
-    _call("fp8q_transpose_blocks", q.data_ptr(), s.data_ptr(), N, K, q.stride(0), qt.data_ptr(),
-          st.data_ptr(), qt.stride(0), _stream(q))
+        _rows(_u8(qt), torch.uint8, "qt", K, N, q.device)
+        _dense(st, torch.float32, "st", (K // 128, N // 128), q.device)
+    _call("fp8q_transpose_blocks", q.data_ptr(), s.data_ptr(), N, K, q.stride(0),
+          _u8(qt).data_ptr(), st.data_ptr(), _u8(qt).stride(0), _stream(q))
     return qt, st
 
 
@@ -176,14 +215,16 @@ def quant_weight_128x128(w: torch.Tensor, pow2: bool = False,
         raise ValueError("w must be contiguous")
     K = w.shape[-1]
     N_all = w.numel() // K if K else 0
+    s_shape = (*w.shape[:-2], w.shape[-2] // 128, K // 128)
     if out is None:
         q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
-        s = torch.empty((*w.shape[:-2], w.shape[-2] // 128, K // 128), dtype=torch.float32,
-                        device=w.device)
+        s = torch.empty(s_shape, dtype=torch.float32, device=w.device)
     else:
         q, s = out
-    _call("fp8q_quant_weight_128x128", w.data_ptr(), N_all, K, K, q.data_ptr(), K, s.data_ptr(),
-          int(bool(pow2)), _stream(w))
+        _dense(_u8(q), torch.uint8, "q", w.shape, w.device)     # row pitch K implied
+        _dense(s, torch.float32, "s", s_shape, w.device)
+    _call("fp8q_quant_weight_128x128", w.data_ptr(), N_all, K, K, _u8(q).data_ptr(), K,
+          s.data_ptr(), int(bool(pow2)), _stream(w))
     return q, s
 
 
@@ -231,6 +272,30 @@ def _workspace(device, nbytes: int) -> torch.Tensor:
     return ws
 
 
+def _dense_gemm_operands(qa, sa, qb, sb, b_rowwise: bool, out, out_dtype):
+    """Checks of the dense GEMMs' operands; returns (qa, qb, out, M, N, K)."""
+    qa, qb = _u8(qa), _u8(qb)
+    _need(qa, torch.uint8, "qa", 2)
+    _need(qb, torch.uint8, "qb", 2)
+    dev = qa.device
+    _same_device(qb, dev, "qb")
+    M, K = qa.shape
+    N = qb.shape[0]
+    if qb.shape[1] != K:
+        raise ValueError("qa and qb disagree on K")
+    _rows(sa, torch.float32, "sa", K // 128, M, dev)             # [K/128, >= M]
+    if b_rowwise:
+        _rows(sb, torch.float32, "sb", K // 128, N, dev)         # [K/128, >= N]
+    else:                                                        # [N/128, K/128], pitch implied
+        _dense(sb, torch.float32, "sb", (-(-N // 128), K // 128), dev)
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=dev)
+    else:
+        _out_code(out.dtype)
+        _rows(out, out.dtype, "out", M, N, dev)
+    return qa, qb, out, M, N, K
+
+
 def gemm_blockscaled(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor,
                      out_dtype=torch.bfloat16, b_rowwise: bool = False,
                      out: Optional[torch.Tensor] = None, split_k: bool = True,
@@ -242,22 +307,13 @@ def gemm_blockscaled(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: t
     ``split_k``: split the last partial wave of tiles along K (uses a device workspace:
     ``workspace`` if given, else a cached per-device buffer).
     """
-    qa, qb = _u8(qa), _u8(qb)
-    _need(qa, torch.uint8, "qa", 2)
-    _need(qb, torch.uint8, "qb", 2)
-    _need(sa, torch.float32, "sa", 2)
-    _need(sb, torch.float32, "sb", 2)
-    M, K = qa.shape
-    N = qb.shape[0]
-    if qb.shape[1] != K:
-        raise ValueError("qa and qb disagree on K")
-    if out is None:
-        out = torch.empty((M, N), dtype=out_dtype, device=qa.device)
+    qa, qb, out, M, N, K = _dense_gemm_operands(qa, sa, qb, sb, b_rowwise, out, out_dtype)
     ws_ptr, ws_len = None, 0
     if split_k and M > 0:
         need = workspace_bytes(M, N, K)
         if need:
             ws = workspace if workspace is not None else _workspace(qa.device, need)
+            _same_device(ws, qa.device, "workspace")
             if ws.numel() * ws.element_size() >= need:
                 ws_ptr, ws_len = ws.data_ptr(), ws.numel() * ws.element_size()
     _call("fp8_gemm_blockscaled_ws", qa.data_ptr(), sa.data_ptr(), sa.stride(0), qb.data_ptr(),
@@ -276,17 +332,7 @@ def gemm_blockscaled_ue8m0(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor,
     [2^-127, 2^127] (the quantizers' ``pow2`` option).  Other scales are reported through
     ``device_error()`` as (8 << 8) | FP8Q_ERR_SCALE.
     """
-    qa, qb = _u8(qa), _u8(qb)
-    _need(qa, torch.uint8, "qa", 2)
-    _need(qb, torch.uint8, "qb", 2)
-    _need(sa, torch.float32, "sa", 2)
-    _need(sb, torch.float32, "sb", 2)
-    M, K = qa.shape
-    N = qb.shape[0]
-    if qb.shape[1] != K:
-        raise ValueError("qa and qb disagree on K")
-    if out is None:
-        out = torch.empty((M, N), dtype=out_dtype, device=qa.device)
+    qa, qb, out, M, N, K = _dense_gemm_operands(qa, sa, qb, sb, b_rowwise, out, out_dtype)
     _call("fp8_gemm_blockscaled_ue8m0", qa.data_ptr(), sa.data_ptr(), sa.stride(0), qb.data_ptr(),
           sb.data_ptr(), sb.stride(0) if b_rowwise else 0,
           BSCALE_ROW if b_rowwise else BSCALE_BLOCK, out.data_ptr(), _out_code(out.dtype),
@@ -305,17 +351,25 @@ def _gemm_grouped(entry: str, qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tens
     qa, qw = _u8(qa), _u8(qw)
     _need(qa, torch.uint8, "qa", 2)
     _need(qw, torch.uint8, "qw", 3)
-    _need(sa, torch.float32, "sa", 2)
-    _need(sw, torch.float32, "sw", 3)
     _need(m_offsets, torch.int32, "m_offsets", 1)
-    if not (qa.is_contiguous() and qw.is_contiguous() and sw.is_contiguous()):
-        raise ValueError("qa, qw and sw must be contiguous")
+    if not (qa.is_contiguous() and qw.is_contiguous()):
+        raise ValueError("qa and qw must be contiguous")
+    dev = qa.device
     M, K = qa.shape
-    E, N, _ = qw.shape
+    E, N, Kw = qw.shape
+    if Kw != K:
+        raise ValueError("qa and qw disagree on K")
+    _same_device(qw, dev, "qw")
+    _same_device(m_offsets, dev, "m_offsets")
+    _rows(sa, torch.float32, "sa", K // 128, M, dev)                          # [K/128, >= sumM]
+    _dense(sw, torch.float32, "sw", (E, -(-N // 128), K // 128), dev)         # [E, N/128, K/128]
     if m_offsets.numel() != E + 1:
         raise ValueError("m_offsets must have E + 1 entries")
     if out is None:
-        out = torch.empty((M, N), dtype=out_dtype, device=qa.device)
+        out = torch.empty((M, N), dtype=out_dtype, device=dev)
+    else:
+        _out_code(out.dtype)
+        _rows(out, out.dtype, "out", M, N, dev)
     _call(entry, qa.data_ptr(), sa.data_ptr(), sa.stride(0), qw.data_ptr(),
           sw.data_ptr(), out.data_ptr(), _out_code(out.dtype), m_offsets.data_ptr(), E, M, N, K,
           _stream(qa))
@@ -346,10 +400,19 @@ def gemm_nopromo(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: torch
     _need(qb, torch.uint8, "qb", 2)
     _need(sa, torch.float32, "sa", 1)
     _need(sb, torch.float32, "sb", 1)
+    dev = qa.device
     M, K = qa.shape
     N = qb.shape[0]
+    if qb.shape[1] != K:
+        raise ValueError("qa and qb disagree on K")
+    for t, name, n in ((qb, "qb", None), (sa, "sa", M), (sb, "sb", N)):
+        _same_device(t, dev, name)
+        if n is not None and t.shape[0] < n:
+            raise ValueError(f"{name} must hold at least {n} scales, got {t.shape[0]}")
     if out is None:
-        out = torch.empty((M, N), dtype=torch.float32, device=qa.device)
+        out = torch.empty((M, N), dtype=torch.float32, device=dev)
+    else:
+        _rows(out, torch.float32, "out", M, N, dev)
     _call("fp8_gemm_nopromo", qa.data_ptr(), sa.data_ptr(), qb.data_ptr(), sb.data_ptr(),
           out.data_ptr(), M, N, K, qa.stride(0), qb.stride(0), out.stride(0), _stream(qa))
     return out
