@@ -259,6 +259,9 @@ def run_gpu(args, rank, world):
         "config": bench_config(w, world),
         "kernels_ms": {"quant_act_1x128": round(ms_act, 5), "quant_weight_128x128": round(ms_w, 5),
                        kernel: round(ms_gemm, 5)},
+        "kernels_ms_stats": {name: _spread(ts) for name, ts in
+                             (("step", t_step), ("quant_act_1x128", t_act),
+                              ("quant_weight_128x128", t_w), (kernel, t_gemm))},
         "gemm_path": path,
         "gemm_paths": paths,
         "gemm_tflops": round(gemm_tflops, 1),
@@ -319,6 +322,12 @@ def run_gpu(args, rank, world):
 
 
 # ------------------------------------------------------------------------------ other workloads
+
+def _spread(ts) -> dict:
+    """Mean, median and best of a list of per-launch times (ms) on this rank."""
+    return {"mean": round(sum(ts) / len(ts), 5), "median": round(statistics.median(ts), 5),
+            "best": round(min(ts), 5)}
+
 
 def _time_ms(fn, reps, flush_l2, warmup=2):
     """Mean device time of fn() over reps, L2 flushed before each (outside the events).

@@ -53,6 +53,11 @@ def test_gemm_path_follows_the_scales():
         bench.gemm_path(SimpleNamespace(gemm="ue8m0"), wgrad)
 
 
+def test_spread_of_per_step_times():
+    got = bench._spread([0.30, 0.10, 0.20, 0.25])
+    assert got == {"mean": 0.2125, "median": 0.225, "best": 0.1}
+
+
 def test_library_ceiling_reports_instead_of_raising():
     """The cuBLASLt FP8 ceiling leg is context only: without a usable GPU it returns an
     'unavailable' entry and the bench line is still printed."""
