@@ -307,9 +307,9 @@ def run_gpu(args, rank, world):
                   "d2h_bytes_per_step": int(C_h.numel() * C_h.element_size()),
                   "ms_per_step": round(ms_e2e, 4), "steps": e2e_steps}
 
-    # ---- parity spot check of this run's output against the oracle (rank 0, 4 rows)
+    # ---- spot check of this run's output against a float64 product of its codes (rank 0)
     if rank == 0 and not args.no_check:
-        res["spot_check"] = spot_check(w, a_bits, b_bits, C)
+        res["spot_check"] = spot_check(w, qA, sA, qW, sW, C)
 
     if rank == 0 and not args.no_configs:
         res["configs"] = config_throughput(fq, flush_l2)
@@ -496,11 +496,10 @@ def library_fp8_ceiling(flush_l2, n: int = 8192, reps: int = 20) -> dict:
 def accumulation_study(fq, rows_sampled=32):
     """Error of the promoted GEMM and of the no-promotion GEMM versus K on the wgrad
     workload (dY [7168, K] x X [2048, K], K = 4096 / 8192 / 16384 prefixes of one draw),
-    against the FP64 oracle on sampled rows.  Promoted: 1x128 codes (and, apples to
-    apples, the 1xK codes with their row scales repeated per group); no-promotion: 1xK
-    codes, one TMEM accumulator over all of K."""
+    against the float64 product of the same codes and scales on sampled rows.  Promoted:
+    1x128 codes (and, apples to apples, the 1xK codes with their row scales repeated per
+    group); no-promotion: 1xK codes, one TMEM accumulator over all of K."""
     import torch
-    import oracle
     w = workloads.wgrad()
     a_full, b_full = w.gen_a(), w.gen_b()
     rows = np.sort(np.random.default_rng(5).choice(w.M, rows_sampled, replace=False))
@@ -528,14 +527,13 @@ def accumulation_study(fq, rows_sampled=32):
                                    sb1.expand(G, -1).contiguous(), out_dtype=torch.float32,
                                    b_rowwise=True)
         torch.cuda.synchronize()
-        # oracle, from the bf16 inputs (never from the GPU's codes)
-        qa_r, sa_r = oracle.quant_act_1x128(a_bits[rows], False)
-        qb_r, sb_r = oracle.quant_act_1x128(b_bits, False)
-        C_ref, T = oracle.gemm_blockscaled_ref(qa_r, sa_r, qb_r, sb_r, b_rowwise=True)
-        qa1_r, sa1_r = oracle.quant_rowwise(a_bits[rows])
-        qb1_r, sb1_r = oracle.quant_rowwise(b_bits)
-        C1_ref, T1 = oracle.gemm_ref(oracle.dequant_rowwise(qa1_r, sa1_r),
-                                     oracle.dequant_rowwise(qb1_r, sb1_r))
+        # float64 products of the codes the GEMMs consumed (1xK row scales repeated per
+        # group give the 1xK codes' exact product)
+        C_ref, T = _fp64_product(qa[rows_t].cpu().numpy(), sa[:, rows_t].cpu().numpy(),
+                                 qb.cpu().numpy(), sb.cpu().numpy(), True)
+        C1_ref, T1 = _fp64_product(qa1[rows_t].cpu().numpy(),
+                                   sa1[rows_t].cpu().numpy()[None, :].repeat(G, 0),
+                                   qb1.cpu().numpy(), sb1.cpu().numpy()[None, :].repeat(G, 0), True)
         res.append({"K": K,
                     "promoted_1x128": stats(C_p[rows_t].cpu().numpy(), C_ref, T),
                     "promoted_1xK_codes": stats(C_p1[rows_t].cpu().numpy(), C1_ref, T1),
@@ -611,16 +609,59 @@ def kernel_rev() -> str:
     return h.hexdigest()[:12]
 
 
-def spot_check(w, a_bits, b_bits, C):
-    import oracle
-    rows = np.array([0, 1, w.M // 2, w.M - 1])
-    qa, sa = oracle.quant_act_1x128(a_bits[rows], w.pow2_a)
-    qb, sb = oracle.quant_weight_128x128(b_bits, w.pow2_b)
-    C_ref, T = oracle.gemm_blockscaled_ref(qa, sa, qb, sb)
+def _e4m3_values() -> np.ndarray:
+    """Float64 value of each of the 256 E4M3 bytes, decoded by torch's float8_e4m3fn."""
     import torch
-    Ch = C[torch.from_numpy(rows).cuda()].float().cpu().numpy().astype(np.float64)
-    ok, fb = oracle.check_bf16(Ch, C_ref, T) if not w.out_fp32 else (oracle.check_fp32(Ch, C_ref, T), None)
-    return {"rows": rows.tolist(), "within_band": bool(ok.all()), "entries": int(ok.size)}
+    return torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def _fp64_product(qa, sa, qb, sb, b_rowwise: bool):
+    """Exact reference for rows of a block-scaled GEMM, from the codes and scales the GPU
+    used: C_ref = sum_k a~ b~ and T = sum_k |a~ b~| in float64, with a~ = E4M3(qa) times
+    its 1x128 scale and b~ likewise (128x128 blocks, or 1x128 along K when b_rowwise).
+    qa uint8 [r, K]; sa float32 [K/128, r]; qb uint8 [N, K]; sb [N/128, K/128] or
+    [K/128, N].  Measurement only: no quantization happens here."""
+    v = _e4m3_values()
+    r, K = qa.shape
+    N, G = qb.shape[0], K // 128
+    A = (v[qa].reshape(r, G, 128) * sa[:G, :r].T.astype(np.float64)[:, :, None]).reshape(r, K)
+    if b_rowwise:
+        B = (v[qb].reshape(N, G, 128) * sb[:G, :N].T.astype(np.float64)[:, :, None]).reshape(N, K)
+    else:
+        B = (v[qb].reshape(N // 128, 128, G, 128)
+             * sb.astype(np.float64)[:, None, :, None]).reshape(N, K)
+    return A @ B.T, np.abs(A) @ np.abs(B).T
+
+
+def _within_band(C, C_ref, T, out_fp32: bool) -> np.ndarray:
+    """The acceptance band of the parity tests: fp32 out within 2e-5 T; bf16 out within one
+    bf16 spacing of C_ref, or (where the sum cancels) within 2e-5 T plus half a bf16
+    spacing of C.  The bf16 spacing at x is float32's spacing times 2^16 (8 against 24
+    significant bits; also right for subnormals)."""
+    C = np.asarray(C, np.float64)
+    d = np.abs(C - C_ref)
+    band = 2e-5 * T + 1e-30
+    if out_fp32:
+        return d <= band
+
+    def spacing(x):
+        return np.spacing(np.abs(x).astype(np.float32)).astype(np.float64) * 65536.0
+
+    return (d <= spacing(C_ref)) | (d <= band + 0.5 * spacing(C))
+
+
+def spot_check(w, qA, sA, qB, sB, C):
+    """Four rows of this run's C (first, second, middle, last) against the float64 product
+    of this run's own codes and scales, in the parity tests' band.  The codes themselves
+    are checked bit for bit against the oracle by the GPU tests."""
+    import torch
+    rows = np.array([0, 1, w.M // 2, w.M - 1])
+    rt = torch.from_numpy(rows).to(C.device)
+    C_ref, T = _fp64_product(qA[rt].cpu().numpy(), sA[:, rt].cpu().numpy(), qB.cpu().numpy(),
+                             sB.cpu().numpy(), w.b_rowwise)
+    ok = _within_band(C[rt].float().cpu().numpy(), C_ref, T, w.out_fp32)
+    return {"rows": rows.tolist(), "within_band": bool(ok.all()), "entries": int(ok.size),
+            "reference": "float64 product of this run's codes and scales"}
 
 
 # ------------------------------------------------------------------------------ CPU oracle

@@ -7,6 +7,7 @@ import subprocess
 import sys
 from types import SimpleNamespace
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -51,6 +52,53 @@ def test_gemm_path_follows_the_scales():
     assert bench.gemm_path(SimpleNamespace(gemm="promoted"), dense) == "promoted"
     with pytest.raises(SystemExit):
         bench.gemm_path(SimpleNamespace(gemm="ue8m0"), wgrad)
+
+
+def test_bench_fp64_reference_agrees_with_the_oracle():
+    """The bench's own float64 product (used by its spot check and accumulation study,
+    which must not call the oracle) against the oracle's reference on oracle codes."""
+    import oracle
+    assert np.array_equal(bench._e4m3_values(), oracle.decode_table(), equal_nan=True)
+    rng = np.random.default_rng(11)
+    a = workloads.normal_bf16(rng, (5, 384), 1.0, 0.01)
+    b = workloads.normal_bf16(rng, (256, 384), 0.02)
+    qa, sa = oracle.quant_act_1x128(a, False)
+    for rowwise in (False, True):
+        qb, sb = oracle.quant_act_1x128(b, True) if rowwise else oracle.quant_weight_128x128(b, False)
+        want, want_T = oracle.gemm_blockscaled_ref(qa, sa, qb, sb, b_rowwise=rowwise)
+        got, got_T = bench._fp64_product(qa, sa, qb, sb, rowwise)
+        assert np.allclose(got, want, rtol=1e-12, atol=0) and np.allclose(got_T, want_T, rtol=1e-12)
+
+
+@pytest.mark.parametrize("out_fp32", [False, True])
+def test_bench_band_is_the_parity_tests_band(out_fp32):
+    import oracle
+    rng = np.random.default_rng(12)
+    C_ref = rng.standard_normal(4000) * np.exp2(rng.integers(-140, 20, 4000))
+    C_ref[:10] = 0.0
+    T = np.abs(C_ref) * np.exp2(rng.uniform(0, 12, 4000))
+    C = C_ref * (1 + rng.standard_normal(4000) * np.exp2(rng.uniform(-30, -4, 4000)))
+    C = C.astype(np.float32).astype(np.float64)
+    want = oracle.check_fp32(C, C_ref, T) if out_fp32 else oracle.check_bf16(C, C_ref, T)[0]
+    got = bench._within_band(C, C_ref, T, out_fp32)
+    assert 0 < got.sum() < got.size
+    assert np.array_equal(got, want)
+
+
+def test_spot_check_on_host_tensors():
+    import oracle
+    import torch
+    w = SimpleNamespace(M=256, b_rowwise=False, out_fp32=False)
+    rng = np.random.default_rng(13)
+    qa, sa = oracle.quant_act_1x128(workloads.normal_bf16(rng, (256, 256), 1.0), False)
+    qb, sb = oracle.quant_weight_128x128(workloads.normal_bf16(rng, (128, 256), 0.02), False)
+    C_ref, _ = oracle.gemm_blockscaled_ref(qa, sa, qb, sb)
+    t = torch.from_numpy
+    C = t(C_ref.astype(np.float32)).to(torch.bfloat16)
+    got = bench.spot_check(w, t(qa), t(sa), t(qb), t(sb), C)
+    assert got["within_band"] and got["entries"] == 4 * 128
+    C[128, 5] += 1.0                                   # a planted error in a checked row
+    assert not bench.spot_check(w, t(qa), t(sa), t(qb), t(sb), C)["within_band"]
 
 
 def test_spread_of_per_step_times():
