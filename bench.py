@@ -493,17 +493,16 @@ def library_fp8_ceiling(flush_l2, n: int = 8192, reps: int = 20) -> dict:
         return {"unavailable": f"{type(e).__name__}: {str(e).splitlines()[0][:200] if str(e) else ''}"}
 
 
-def accumulation_study(fq, rows_sampled=32):
+def accumulation_study(fq, rows_sampled=32, w=None, ks=(4096, 8192, 16384)):
     """Error of the promoted GEMM and of the no-promotion GEMM versus K on the wgrad
     workload (dY [7168, K] x X [2048, K], K = 4096 / 8192 / 16384 prefixes of one draw),
     against the float64 product of the same codes and scales on sampled rows.  Promoted:
     1x128 codes (and, apples to apples, the 1xK codes with their row scales repeated per
     group); no-promotion: 1xK codes, one TMEM accumulator over all of K."""
     import torch
-    w = workloads.wgrad()
+    w = workloads.wgrad() if w is None else w
     a_full, b_full = w.gen_a(), w.gen_b()
     rows = np.sort(np.random.default_rng(5).choice(w.M, rows_sampled, replace=False))
-    rows_t = torch.from_numpy(rows).cuda()
     res = []
 
     def stats(Cs, C_ref, T):
@@ -512,10 +511,11 @@ def accumulation_study(fq, rows_sampled=32):
         return {"max_rel_T": float(r.max()), "median_rel_T": float(np.median(r)),
                 "rel_frobenius": float(np.linalg.norm(d) / np.linalg.norm(C_ref))}
 
-    for K in (4096, 8192, 16384):
+    for K in ks:
         a_bits = np.ascontiguousarray(a_full[:, :K])
         b_bits = np.ascontiguousarray(b_full[:, :K])
         A, B = dev_bf16(a_bits), dev_bf16(b_bits)
+        rows_t = torch.from_numpy(rows).to(A.device)
         G = K // 128
         qa, sa = fq.quant_act_1x128(A, False)
         qb, sb = fq.quant_act_1x128(B, False)

@@ -101,6 +101,47 @@ def test_spot_check_on_host_tensors():
     assert not bench.spot_check(w, t(qa), t(sa), t(qb), t(sb), C)["within_band"]
 
 
+def test_accumulation_study_runs_on_host_stand_ins(monkeypatch):
+    """The accumulation study's plumbing (row sampling, scale layouts, the float64 products
+    of the same codes) on a small workload, with the library replaced by oracle-backed
+    host stand-ins whose GEMMs are the exact product rounded to fp32: every reported
+    error is then at fp32 rounding level."""
+    import oracle
+    import torch
+    t = torch.from_numpy
+    v = oracle.decode_table()
+
+    def bits(x):
+        return x.view(torch.int16).numpy().view(np.uint16)
+
+    def gemm_blockscaled(qa, sa, qb, sb, out_dtype, b_rowwise):
+        C, _ = bench._fp64_product(qa.numpy(), sa.numpy(), qb.numpy(), sb.numpy(), b_rowwise)
+        return t(C.astype(np.float32))
+
+    def gemm_nopromo(qa, sa, qb, sb):
+        A = v[qa.numpy()] * sa.numpy().astype(np.float64)[:, None]
+        B = v[qb.numpy()] * sb.numpy().astype(np.float64)[:, None]
+        return t((A @ B.T).astype(np.float32))
+
+    fake = SimpleNamespace(
+        quant_act_1x128=lambda x, pow2: tuple(map(t, oracle.quant_act_1x128(bits(x), pow2))),
+        quant_rowwise=lambda x: tuple(map(t, oracle.quant_rowwise(bits(x)))),
+        gemm_blockscaled=gemm_blockscaled, gemm_nopromo=gemm_nopromo)
+    monkeypatch.setattr(bench, "dev_bf16",
+                        lambda b: t(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16))
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    rng = np.random.default_rng(14)
+    a = workloads.normal_bf16(rng, (96, 512), 1e-3)
+    b = workloads.normal_bf16(rng, (256, 512), 1.0)
+    w = SimpleNamespace(M=96, gen_a=lambda: a, gen_b=lambda: b)
+    res = bench.accumulation_study(fake, rows_sampled=8, w=w, ks=(256, 512))
+    assert res["rows_sampled"] == 8 and [r["K"] for r in res["results"]] == [256, 512]
+    for r in res["results"]:
+        for key in ("promoted_1x128", "promoted_1xK_codes", "no_promotion_1xK_codes"):
+            assert 0 <= r[key]["max_rel_T"] < 1e-7 and r[key]["rel_frobenius"] < 1e-6
+    json.dumps(res)
+
+
 def test_spread_of_per_step_times():
     got = bench._spread([0.30, 0.10, 0.20, 0.25])
     assert got == {"mean": 0.2125, "median": 0.225, "best": 0.1}
