@@ -650,15 +650,16 @@ def _within_band(C, C_ref, T, out_fp32: bool) -> np.ndarray:
     return (d <= spacing(C_ref)) | (d <= band + 0.5 * spacing(C))
 
 
-def spot_check(w, qA, sA, qB, sB, C):
+def spot_check(w, qA, sA, qB, sB, C, b_rowwise: bool = False):
     """Four rows of this run's C (first, second, middle, last) against the float64 product
     of this run's own codes and scales, in the parity tests' band.  The codes themselves
-    are checked bit for bit against the oracle by the GPU tests."""
+    are checked bit for bit against the oracle by the GPU tests.  b_rowwise: the B scale
+    mode the GEMM ran with (the timed step always uses 128x128 weight blocks)."""
     import torch
     rows = np.array([0, 1, w.M // 2, w.M - 1])
     rt = torch.from_numpy(rows).to(C.device)
     C_ref, T = _fp64_product(qA[rt].cpu().numpy(), sA[:, rt].cpu().numpy(), qB.cpu().numpy(),
-                             sB.cpu().numpy(), w.b_rowwise)
+                             sB.cpu().numpy(), b_rowwise)
     ok = _within_band(C[rt].float().cpu().numpy(), C_ref, T, w.out_fp32)
     return {"rows": rows.tolist(), "within_band": bool(ok.all()), "entries": int(ok.size),
             "reference": "float64 product of this run's codes and scales"}

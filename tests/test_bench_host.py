@@ -88,7 +88,7 @@ def test_bench_band_is_the_parity_tests_band(out_fp32):
 def test_spot_check_on_host_tensors():
     import oracle
     import torch
-    w = SimpleNamespace(M=256, b_rowwise=False, out_fp32=False)
+    w = SimpleNamespace(M=256, b_rowwise=True, out_fp32=False)   # the step's mode wins
     rng = np.random.default_rng(13)
     qa, sa = oracle.quant_act_1x128(workloads.normal_bf16(rng, (256, 256), 1.0), False)
     qb, sb = oracle.quant_weight_128x128(workloads.normal_bf16(rng, (128, 256), 0.02), False)
@@ -99,6 +99,12 @@ def test_spot_check_on_host_tensors():
     assert got["within_band"] and got["entries"] == 4 * 128
     C[128, 5] += 1.0                                   # a planted error in a checked row
     assert not bench.spot_check(w, t(qa), t(sa), t(qb), t(sb), C)["within_band"]
+    # ROW-mode B scales (1x128 along K), as a caller with a Wgrad-style GEMM passes them
+    qb_r, sb_r = oracle.quant_act_1x128(workloads.normal_bf16(rng, (128, 256), 1.0), False)
+    C_r, _ = oracle.gemm_blockscaled_ref(qa, sa, qb_r, sb_r, b_rowwise=True)
+    got = bench.spot_check(SimpleNamespace(M=256, out_fp32=True), t(qa), t(sa), t(qb_r), t(sb_r),
+                           t(C_r.astype(np.float32)), b_rowwise=True)
+    assert got["within_band"]
 
 
 def test_accumulation_study_runs_on_host_stand_ins(monkeypatch):
