@@ -42,6 +42,46 @@ def test_library_exports_every_declared_symbol(L):
         assert name in fq.SIGNATURES, f"binding lacks {name}"
 
 
+def declarations():
+    """name -> (return type, [parameter types]) of every function the header declares."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for ret, name, params in re.findall(
+            r"((?:const\s+)?[A-Za-z_]\w*\s*\**)\s*\b((?:fp8q|fp8)_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", src):
+        ps = [] if params.strip() in ("", "void") else [p.strip() for p in params.split(",")]
+        types = [re.sub(r"\s*\b\w+$", "", p) if not p.endswith("*") else p for p in ps]
+        out[name] = (ret.strip(), types)
+    return out
+
+
+def _ctype_of(c_type: str):
+    c = " ".join(c_type.replace("*", " * ").split())
+    if c == "size_t *":
+        return ctypes.POINTER(ctypes.c_size_t)
+    if c in ("const char *",):
+        return ctypes.c_char_p
+    if "*" in c:
+        return ctypes.c_void_p
+    return {"int": ctypes.c_int, "int64_t": ctypes.c_int64, "uint64_t": ctypes.c_uint64,
+            "size_t": ctypes.c_size_t, "float": ctypes.c_float}[c]
+
+
+def test_binding_signatures_match_the_header():
+    """Every ctypes signature in the binding has the header's arity and argument widths:
+    a mismatch would pass garbage pointers or sizes into the library."""
+    import fp8_fine_grained_weight_b200 as fq
+    decl = declarations()
+    assert set(decl) == set(declared_functions())
+    for name, (ret, params) in decl.items():
+        res, args = fq.SIGNATURES[name]
+        assert res is _ctype_of(ret), (name, ret)
+        want = [_ctype_of(p) for p in params]
+        assert len(args) == len(want), (name, len(args), len(want))
+        for i, (got, w) in enumerate(zip(args, want)):
+            same = got is w or (getattr(got, "_type_", None) is getattr(w, "_type_", 0))
+            assert same, (name, i, params[i], got, w)
+
+
 def test_status_strings_and_version(L):
     assert L.fp8q_abi_version() == 1
     assert L.fp8q_status_string(0) == b"ok"
