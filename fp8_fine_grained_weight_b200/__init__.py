@@ -261,10 +261,11 @@ def workspace_bytes(M: int, N: int, K: int) -> int:
     return int(n.value)
 
 
-def _workspace(device, nbytes: int) -> torch.Tensor:
-    """A per-device scratch buffer of at least nbytes, grown on demand (never shrunk).
-    Calls on one stream reuse it; concurrent streams should pass their own."""
-    key = torch.device(device).index
+def _workspace(device, stream: int, nbytes: int) -> torch.Tensor:
+    """A scratch buffer of at least nbytes for one (device, stream), grown on demand
+    (never shrunk).  Calls on one stream run in order and share it; GEMMs on different
+    streams get different buffers, so they may run concurrently."""
+    key = (torch.device(device).index, int(stream))
     ws = _WORKSPACE.get(key)
     if ws is None or ws.numel() < nbytes:
         ws = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
@@ -305,14 +306,14 @@ def gemm_blockscaled(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: t
     qa uint8 [M, K]; sa fp32 [K/128, >= M]; qb uint8 [N, K];
     sb fp32 [N/128, K/128] (128x128 blocks) or, with ``b_rowwise``, [K/128, >= N].
     ``split_k``: split the last partial wave of tiles along K (uses a device workspace:
-    ``workspace`` if given, else a cached per-device buffer).
+    ``workspace`` if given, else a buffer cached per device and stream).
     """
     qa, qb, out, M, N, K = _dense_gemm_operands(qa, sa, qb, sb, b_rowwise, out, out_dtype)
     ws_ptr, ws_len = None, 0
     if split_k and M > 0:
         need = workspace_bytes(M, N, K)
         if need:
-            ws = workspace if workspace is not None else _workspace(qa.device, need)
+            ws = workspace if workspace is not None else _workspace(qa.device, _stream(qa), need)
             _same_device(ws, qa.device, "workspace")
             if ws.numel() * ws.element_size() >= need:
                 ws_ptr, ws_len = ws.data_ptr(), ws.numel() * ws.element_size()

@@ -156,3 +156,23 @@ def test_fp8_linear_wiring(calls, pow2):
                                      "fp8q_quant_act_dual", "fp8q_transpose_blocks", gemm, gemm]
     # Wgrad: B scales in ROW mode (mode argument 1) with the transposed copy's pitch K
     assert calls[-1][1][6] == fq.BSCALE_ROW and calls[-1][1][5] == K
+
+
+def test_split_workspace_is_per_stream(calls, monkeypatch):
+    """The cached split-K workspace is keyed by (device, stream): GEMMs on one stream share
+    it (they run in order), GEMMs on different streams never do."""
+    monkeypatch.setattr(fq, "workspace_bytes", lambda M, N, K: 4096)
+    monkeypatch.setattr(fq, "_WORKSPACE", {})
+    qa, sa, qb, sb = E(256, 384), E(3, 256, dtype=f32), E(512, 384), E(4, 3, dtype=f32)
+    ptrs = []
+    for stream in (11, 11, 22):
+        monkeypatch.setattr(fq, "_stream", lambda t, s=stream: s)
+        fq.gemm_blockscaled(qa, sa, qb, sb)
+        name, args = calls[-1]
+        assert name == "fp8_gemm_blockscaled_ws" and args[-1] == stream and args[-2] >= 4096
+        ptrs.append(args[-3])
+    assert ptrs[0] == ptrs[1] != ptrs[2]
+    own = E(8192)
+    fq.gemm_blockscaled(qa, sa, qb, sb, workspace=own)       # a caller's buffer is used as is
+    assert calls[-1][1][-3] == own.data_ptr()
+
