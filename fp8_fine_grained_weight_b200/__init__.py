@@ -13,6 +13,8 @@ Layouts (see include/fp8q.h):
 """
 from __future__ import annotations
 
+import collections
+import contextlib
 import ctypes
 import os
 from typing import Optional, Tuple
@@ -93,6 +95,13 @@ def _stream(t: torch.Tensor) -> int:
     return torch.cuda.current_stream(t.device).cuda_stream
 
 
+def _on(t: torch.Tensor):
+    """Make t's device the current one for a library call.  The library sizes grids and
+    binds its driver context through the current device, so operands on another GPU must
+    not be passed while a different device is current."""
+    return torch.cuda.device(t.device) if t.is_cuda else contextlib.nullcontext()
+
+
 def _require_cuda(t: torch.Tensor, name: str) -> None:
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA tensor")
@@ -156,8 +165,9 @@ def quant_act_1x128(x: torch.Tensor, pow2: bool = False, ld_scale: Optional[int]
         ld = s.stride(0)
         if ld_scale is not None and int(ld_scale) != ld:
             raise ValueError(f"ld_scale {ld_scale} disagrees with the row stride {ld} of s")
-    _call("fp8q_quant_act_1x128", x.data_ptr(), M, K, x.stride(0), _u8(q).data_ptr(),
-          _u8(q).stride(0), s.data_ptr(), ld, int(bool(pow2)), _stream(x))
+    with _on(x):
+        _call("fp8q_quant_act_1x128", x.data_ptr(), M, K, x.stride(0), _u8(q).data_ptr(),
+              _u8(q).stride(0), s.data_ptr(), ld, int(bool(pow2)), _stream(x))
     return q, s
 
 
@@ -179,9 +189,10 @@ def quant_act_dual(x: torch.Tensor, pow2: bool = False, out=None):
         _rows(_u8(qt), torch.uint8, "qt", K, M, x.device)
         _rows(st, torch.float32, "st", M // 128, K, x.device)
     q8, qt8 = _u8(q), _u8(qt)
-    _call("fp8q_quant_act_dual", x.data_ptr(), M, K, x.stride(0), q8.data_ptr(), q8.stride(0),
-          s.data_ptr(), s.stride(0), qt8.data_ptr(), qt8.stride(0), st.data_ptr(), st.stride(0),
-          int(bool(pow2)), _stream(x))
+    with _on(x):
+        _call("fp8q_quant_act_dual", x.data_ptr(), M, K, x.stride(0), q8.data_ptr(), q8.stride(0),
+              s.data_ptr(), s.stride(0), qt8.data_ptr(), qt8.stride(0), st.data_ptr(), st.stride(0),
+              int(bool(pow2)), _stream(x))
     return q, s, qt, st
 
 
@@ -200,8 +211,9 @@ def transpose_blocks(q: torch.Tensor, s: torch.Tensor, out=None):
         qt, st = out
         _rows(_u8(qt), torch.uint8, "qt", K, N, q.device)
         _dense(st, torch.float32, "st", (K // 128, N // 128), q.device)
-    _call("fp8q_transpose_blocks", q.data_ptr(), s.data_ptr(), N, K, q.stride(0),
-          _u8(qt).data_ptr(), st.data_ptr(), _u8(qt).stride(0), _stream(q))
+    with _on(q):
+        _call("fp8q_transpose_blocks", q.data_ptr(), s.data_ptr(), N, K, q.stride(0),
+              _u8(qt).data_ptr(), st.data_ptr(), _u8(qt).stride(0), _stream(q))
     return qt, st
 
 
@@ -223,8 +235,9 @@ def quant_weight_128x128(w: torch.Tensor, pow2: bool = False,
         q, s = out
         _dense(_u8(q), torch.uint8, "q", w.shape, w.device)     # row pitch K implied
         _dense(s, torch.float32, "s", s_shape, w.device)
-    _call("fp8q_quant_weight_128x128", w.data_ptr(), N_all, K, K, _u8(q).data_ptr(), K,
-          s.data_ptr(), int(bool(pow2)), _stream(w))
+    with _on(w):
+        _call("fp8q_quant_weight_128x128", w.data_ptr(), N_all, K, K, _u8(q).data_ptr(), K,
+              s.data_ptr(), int(bool(pow2)), _stream(w))
     return q, s
 
 
@@ -234,8 +247,9 @@ def quant_rowwise(x: torch.Tensor, pow2: bool = False):
     M, K = x.shape
     q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
     s = torch.empty((M,), dtype=torch.float32, device=x.device)
-    _call("fp8q_quant_rowwise", x.data_ptr(), M, K, x.stride(0), q.data_ptr(), q.stride(0),
-          s.data_ptr(), int(bool(pow2)), _stream(x))
+    with _on(x):
+        _call("fp8q_quant_rowwise", x.data_ptr(), M, K, x.stride(0), q.data_ptr(), q.stride(0),
+              s.data_ptr(), int(bool(pow2)), _stream(x))
     return q, s
 
 
@@ -251,7 +265,14 @@ def _out_code(out_dtype) -> int:
     raise TypeError("out_dtype must be torch.bfloat16 or torch.float32")
 
 
-_WORKSPACE = {}
+# Split-K workspaces cached per (device, stream), least recently used first.  At most
+# _WORKSPACE_MAX are kept (each at most a few tens of MB); a program that cycles through
+# more streams than that gets a new buffer when it returns to an evicted one.  A buffer is
+# allocated on, and only ever used by, its own stream, so dropping it is safe while GEMMs on
+# that stream are still in flight (the caching allocator orders the reuse after them).
+# Callers that want no cached buffers pass workspace= themselves.
+_WORKSPACE: "collections.OrderedDict" = collections.OrderedDict()
+_WORKSPACE_MAX = 8
 
 
 def workspace_bytes(M: int, N: int, K: int) -> int:
@@ -270,6 +291,9 @@ def _workspace(device, stream: int, nbytes: int) -> torch.Tensor:
     if ws is None or ws.numel() < nbytes:
         ws = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
         _WORKSPACE[key] = ws
+    _WORKSPACE.move_to_end(key)
+    while len(_WORKSPACE) > _WORKSPACE_MAX:
+        _WORKSPACE.popitem(last=False)
     return ws
 
 
@@ -310,17 +334,18 @@ def gemm_blockscaled(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: t
     """
     qa, qb, out, M, N, K = _dense_gemm_operands(qa, sa, qb, sb, b_rowwise, out, out_dtype)
     ws_ptr, ws_len = None, 0
-    if split_k and M > 0:
-        need = workspace_bytes(M, N, K)
-        if need:
-            ws = workspace if workspace is not None else _workspace(qa.device, _stream(qa), need)
-            _same_device(ws, qa.device, "workspace")
-            if ws.numel() * ws.element_size() >= need:
-                ws_ptr, ws_len = ws.data_ptr(), ws.numel() * ws.element_size()
-    _call("fp8_gemm_blockscaled_ws", qa.data_ptr(), sa.data_ptr(), sa.stride(0), qb.data_ptr(),
-          sb.data_ptr(), sb.stride(0) if b_rowwise else 0,
-          BSCALE_ROW if b_rowwise else BSCALE_BLOCK, out.data_ptr(), _out_code(out.dtype),
-          M, N, K, qa.stride(0), qb.stride(0), out.stride(0), ws_ptr, ws_len, _stream(qa))
+    with _on(qa):
+        if split_k and M > 0:
+            need = workspace_bytes(M, N, K)
+            if need:
+                ws = workspace if workspace is not None else _workspace(qa.device, _stream(qa), need)
+                _same_device(ws, qa.device, "workspace")
+                if ws.numel() * ws.element_size() >= need:
+                    ws_ptr, ws_len = ws.data_ptr(), ws.numel() * ws.element_size()
+        _call("fp8_gemm_blockscaled_ws", qa.data_ptr(), sa.data_ptr(), sa.stride(0), qb.data_ptr(),
+              sb.data_ptr(), sb.stride(0) if b_rowwise else 0,
+              BSCALE_ROW if b_rowwise else BSCALE_BLOCK, out.data_ptr(), _out_code(out.dtype),
+              M, N, K, qa.stride(0), qb.stride(0), out.stride(0), ws_ptr, ws_len, _stream(qa))
     return out
 
 
@@ -334,10 +359,11 @@ def gemm_blockscaled_ue8m0(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor,
     ``device_error()`` as (8 << 8) | FP8Q_ERR_SCALE.
     """
     qa, qb, out, M, N, K = _dense_gemm_operands(qa, sa, qb, sb, b_rowwise, out, out_dtype)
-    _call("fp8_gemm_blockscaled_ue8m0", qa.data_ptr(), sa.data_ptr(), sa.stride(0), qb.data_ptr(),
-          sb.data_ptr(), sb.stride(0) if b_rowwise else 0,
-          BSCALE_ROW if b_rowwise else BSCALE_BLOCK, out.data_ptr(), _out_code(out.dtype),
-          M, N, K, qa.stride(0), qb.stride(0), out.stride(0), _stream(qa))
+    with _on(qa):
+        _call("fp8_gemm_blockscaled_ue8m0", qa.data_ptr(), sa.data_ptr(), sa.stride(0), qb.data_ptr(),
+              sb.data_ptr(), sb.stride(0) if b_rowwise else 0,
+              BSCALE_ROW if b_rowwise else BSCALE_BLOCK, out.data_ptr(), _out_code(out.dtype),
+              M, N, K, qa.stride(0), qb.stride(0), out.stride(0), _stream(qa))
     return out
 
 
@@ -371,9 +397,10 @@ def _gemm_grouped(entry: str, qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tens
     else:
         _out_code(out.dtype)
         _rows(out, out.dtype, "out", M, N, dev)
-    _call(entry, qa.data_ptr(), sa.data_ptr(), sa.stride(0), qw.data_ptr(),
-          sw.data_ptr(), out.data_ptr(), _out_code(out.dtype), m_offsets.data_ptr(), E, M, N, K,
-          _stream(qa))
+    with _on(qa):
+        _call(entry, qa.data_ptr(), sa.data_ptr(), sa.stride(0), qw.data_ptr(),
+              sw.data_ptr(), out.data_ptr(), _out_code(out.dtype), m_offsets.data_ptr(), E, M, N, K,
+              _stream(qa))
     return out
 
 
@@ -414,14 +441,18 @@ def gemm_nopromo(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: torch
         out = torch.empty((M, N), dtype=torch.float32, device=dev)
     else:
         _rows(out, torch.float32, "out", M, N, dev)
-    _call("fp8_gemm_nopromo", qa.data_ptr(), sa.data_ptr(), qb.data_ptr(), sb.data_ptr(),
-          out.data_ptr(), M, N, K, qa.stride(0), qb.stride(0), out.stride(0), _stream(qa))
+    with _on(qa):
+        _call("fp8_gemm_nopromo", qa.data_ptr(), sa.data_ptr(), qb.data_ptr(), sb.data_ptr(),
+              out.data_ptr(), M, N, K, qa.stride(0), qb.stride(0), out.stride(0), _stream(qa))
     return out
 
 
 def device_error(device=None) -> int:
-    """Read and clear the library's device error word (synchronizes the current stream)."""
-    return int(lib().fp8q_get_device_error(torch.cuda.current_stream(device).cuda_stream))
+    """Read and clear the library's device error word on `device` (default: the current
+    device); synchronizes that device's current stream."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        return int(lib().fp8q_get_device_error(torch.cuda.current_stream(dev).cuda_stream))
 
 
 def status_string(status: int) -> str:

@@ -16,8 +16,14 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfp8q.so")
 SOURCES = [os.path.join(CSRC, "fp8q.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "quant.cuh", "gemm.cuh")] + [
-    os.path.join(ROOT, "include", "fp8q.h")]
+
+
+def deps() -> list:
+    """Every file the library is built from: the sources, every header under csrc/ and the
+    public header.  A change to any of them makes the next build() recompile."""
+    hdrs = sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h")))
+    return SOURCES + hdrs + [os.path.join(ROOT, "include", "fp8q.h")]
+
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -38,7 +44,7 @@ def command(out: str = LIB, extra=()) -> list:
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and os.path.exists(LIB):
         t = os.path.getmtime(LIB)
-        if all(os.path.getmtime(d) <= t for d in DEPS):
+        if all(os.path.getmtime(d) <= t for d in deps()):
             return LIB
     tmp = LIB + ".tmp"
     res = subprocess.run(command(tmp), capture_output=True, text=True)

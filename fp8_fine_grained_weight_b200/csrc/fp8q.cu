@@ -63,34 +63,17 @@ int encode_operand(CUtensorMap* tm, const void* base, uint64_t K, uint64_t rows,
   return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
-// Tile shape of the promoted GEMMs: one CTA per 128 x 256 tile, two 256-column TMEM
-// accumulator buffers.  The kernel template also has a CTA-pair shape (cta_group::2,
-// 256 x 128 tiles, four 128-column buffers per CTA); it passed the same parity tests but
-// measured slower on every promoted workload (dense 4096 x 7168 x 7168: 0.34 ms against
-// 0.24 ms: its groups are half as large, so the per-group hand-off is paid twice as
-// often), and the launcher does not instantiate it.
-constexpr bool kPair = false;
-using Cfg1 = fp8q::GemmCfg<kPair>;
+// Tile shape of the promoted GEMMs: one CTA per 128 x 256 tile (the same shape for both
+// B scale modes).
+using Cfg1 = fp8q::GemmCfg<false>;
 
-template <bool PAIR, bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16>
+template <bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16>
 struct GemmLauncher {
-  using Cfg = fp8q::GemmCfg<PAIR>;
-  static constexpr auto kern = fp8q::gemm_fp8_blockscaled_kernel<PAIR, PROMOTE, ROW_B, GROUPED, OUT_BF16>;
+  using Cfg = fp8q::GemmCfg<ROW_B>;
+  static constexpr auto kern = fp8q::gemm_fp8_blockscaled_kernel<PROMOTE, ROW_B, GROUPED, OUT_BF16>;
 
-  static void config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, cudaStream_t stream) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = Cfg::kCG;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.blockDim = dim3(fp8q::kGemmThreads);
-    cfg.dynamicSmemBytes = Cfg::smem_bytes;
-    cfg.stream = stream;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-  }
-
-  // Co-resident units (CTAs, or CTA pairs) on the current device; sets the kernel's
-  // attributes on first use.  0 on failure.
+  // Co-resident CTAs on the current device; sets the kernel's attributes on first use.
+  // 0 on failure.
   static int max_units() {
     static std::atomic<int> cached[64];
     int dev = 0;
@@ -100,32 +83,23 @@ struct GemmLauncher {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(Cfg::smem_bytes)) != cudaSuccess)
       return 0;
-    if (Cfg::kCG > 1 &&
-        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess)
-      return 0;
-    int sms = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    config(cfg, attr, nullptr);
-    cfg.gridDim = dim3(static_cast<unsigned>(sms / Cfg::kCG * Cfg::kCG));
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+    int sms = 0, per_sm = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, fp8q::kGemmThreads,
+                                                      Cfg::smem_bytes) != cudaSuccess ||
+        per_sm <= 0) {
       (void)cudaGetLastError();   // the query's failure is handled here, not by the next launch check
-      n = sms / Cfg::kCG;
+      return 0;
     }
-    cached[dev].store(n, std::memory_order_release);
-    return n;
+    units = sms * per_sm;
+    cached[dev].store(units, std::memory_order_release);
+    return units;
   }
 
   static int launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& args,
-                    int64_t grid_units, cudaStream_t stream) {
-    if (grid_units <= 0) return FP8Q_OK;
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    config(cfg, attr, stream);
-    cfg.gridDim = dim3(static_cast<unsigned>(grid_units * Cfg::kCG));
-    if (cudaLaunchKernelEx(&cfg, kern, tmA, tmB, args) != cudaSuccess) return FP8Q_ERR_CUDA;
+                    int64_t grid, cudaStream_t stream) {
+    if (grid <= 0) return FP8Q_OK;
+    kern<<<static_cast<unsigned>(grid), fp8q::kGemmThreads, Cfg::smem_bytes, stream>>>(tmA, tmB, args);
     return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
   }
 };
@@ -138,9 +112,7 @@ struct SplitPlan {
   size_t ws_bytes;
 };
 
-template <bool PAIR>
 SplitPlan plan_split(int64_t tiles, int64_t G, int64_t units) {
-  using Cfg = fp8q::GemmCfg<PAIR>;
   SplitPlan sp{tiles, 0, 1, tiles < units ? tiles : units, 0};
   if (units <= 0) return sp;
   const int64_t full_waves = tiles / units, tail = tiles % units;
@@ -152,7 +124,7 @@ SplitPlan plan_split(int64_t tiles, int64_t G, int64_t units) {
   sp.tail_tiles = tail;
   sp.tail_split = split;
   sp.grid_units = full_waves > 0 ? units : tail * split;
-  sp.ws_bytes = static_cast<size_t>(tail * split) * Cfg::kTileM * Cfg::kN * sizeof(float);
+  sp.ws_bytes = static_cast<size_t>(tail * split) * Cfg1::kTileM * Cfg1::kN * sizeof(float);
   return sp;
 }
 
@@ -171,14 +143,29 @@ int check_gemm_common(const uint8_t* A, const uint8_t* B, const void* C, int out
   return FP8Q_OK;
 }
 
+// Host checks of the dense block-scaled GEMMs' arguments (everything but a workspace).
+int check_dense_blockscaled(const uint8_t* A, const float* sA, int64_t ld_sa, const uint8_t* B,
+                            const float* sB, int64_t ld_sb, int b_scale_mode, const void* C,
+                            int out_dtype, int64_t M, int64_t N, int64_t K, int64_t lda,
+                            int64_t ldb, int64_t ldc) {
+  int st = check_gemm_common(A, B, C, out_dtype, M, N, K, lda, ldb, ldc);
+  if (st != FP8Q_OK) return st;
+  if (!sA || !sB) return FP8Q_ERR_NULL;
+  if (b_scale_mode != FP8Q_BSCALE_BLOCK128x128 && b_scale_mode != FP8Q_BSCALE_ROW1x128)
+    return FP8Q_ERR_UNSUPPORTED;
+  if (ld_sa < M) return FP8Q_ERR_SHAPE;
+  if (b_scale_mode == FP8Q_BSCALE_ROW1x128 && ld_sb < N) return FP8Q_ERR_SHAPE;
+  if (!aligned(sA, 4) || !aligned(sB, 4)) return FP8Q_ERR_ALIGN;
+  return FP8Q_OK;
+}
+
 // Launch one GEMM instantiation.  work: tiles (a bound for grouped).  Dense GEMMs given a
 // large enough workspace split their last partial wave along K and finish with a
 // reduction launch on the same stream.
-template <bool PAIR, bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16>
+template <bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16>
 int run_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, GemmArgs a, int64_t work,
              void* ws, size_t ws_bytes, cudaStream_t st) {
-  using L = GemmLauncher<PAIR, PROMOTE, ROW_B, GROUPED, OUT_BF16>;
-  using Cfg = fp8q::GemmCfg<PAIR>;
+  using L = GemmLauncher<PROMOTE, ROW_B, GROUPED, OUT_BF16>;
   const int units = L::max_units();
   if (units <= 0) return FP8Q_ERR_CUDA;
   a.ws = nullptr;
@@ -187,7 +174,7 @@ int run_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, GemmArgs a, int64_t
   a.tail_split = 1;
   int64_t grid = work < units ? work : units;
   if (!GROUPED && PROMOTE && ws != nullptr) {
-    const SplitPlan sp = plan_split<PAIR>(work, a.G, units);
+    const SplitPlan sp = plan_split(work, a.G, units);
     if (sp.tail_tiles > 0 && sp.ws_bytes <= ws_bytes) {
       a.ws = static_cast<float*>(ws);
       a.tiles_full = static_cast<int>(sp.tiles_full);
@@ -198,28 +185,25 @@ int run_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, GemmArgs a, int64_t
   }
   int st_code = L::launch(tmA, tmB, a, grid, st);
   if (st_code != FP8Q_OK || a.tail_tiles == 0) return st_code;
-  const int mt_total = static_cast<int>((a.M + Cfg::kTileM - 1) / Cfg::kTileM);
-  fp8q::splitk_reduce_kernel<OUT_BF16, Cfg::kTileM, Cfg::kN>
-      <<<a.tail_tiles * Cfg::kTileM, Cfg::kN, 0, st>>>(a, mt_total);
+  const int mt_total = static_cast<int>((a.M + Cfg1::kTileM - 1) / Cfg1::kTileM);
+  fp8q::splitk_reduce_kernel<OUT_BF16, Cfg1::kTileM, Cfg1::kN>
+      <<<a.tail_tiles * Cfg1::kTileM, Cfg1::kN, 0, st>>>(a, mt_total);
   return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
-// Promoted dense GEMM: tile shape, B scale mode and output type chosen at run time.
-template <bool PAIR>
+// Promoted dense GEMM: B scale mode and output type chosen at run time.
 int dispatch_dense(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, bool row_b,
                    bool bf16, int64_t work, void* ws, size_t ws_bytes, cudaStream_t st) {
   if (row_b) {
-    return bf16 ? run_gemm<PAIR, true, true, false, true>(tmA, tmB, a, work, ws, ws_bytes, st)
-                : run_gemm<PAIR, true, true, false, false>(tmA, tmB, a, work, ws, ws_bytes, st);
+    return bf16 ? run_gemm<true, true, false, true>(tmA, tmB, a, work, ws, ws_bytes, st)
+                : run_gemm<true, true, false, false>(tmA, tmB, a, work, ws, ws_bytes, st);
   }
-  return bf16 ? run_gemm<PAIR, true, false, false, true>(tmA, tmB, a, work, ws, ws_bytes, st)
-              : run_gemm<PAIR, true, false, false, false>(tmA, tmB, a, work, ws, ws_bytes, st);
+  return bf16 ? run_gemm<true, false, false, true>(tmA, tmB, a, work, ws, ws_bytes, st)
+              : run_gemm<true, false, false, false>(tmA, tmB, a, work, ws, ws_bytes, st);
 }
 
-template <bool PAIR>
 int64_t dense_tiles(int64_t M, int64_t N) {
-  using Cfg = fp8q::GemmCfg<PAIR>;
-  return ((M + Cfg::kTileM - 1) / Cfg::kTileM) * ((N + Cfg::kN - 1) / Cfg::kN);
+  return ((M + Cfg1::kTileM - 1) / Cfg1::kTileM) * ((N + Cfg1::kN - 1) / Cfg1::kN);
 }
 
 static_assert(fp8q::kErrScale == FP8Q_ERR_SCALE, "device status code of a bad scale");
@@ -276,8 +260,8 @@ __global__ void selftest_wait_kernel(uint64_t timeout_ns) {
 // callbacks that must not re-enter the allocator, or runtimes that forbid cudaMalloc
 // on their hot path.  For them the split-K workspace lives in this file-scope device
 // array instead of a caller buffer.  It is sized for the largest split plan on a 148-SM
-// B200 (at most one 128 x 256 FP32 partial tile per SM), and every GPU that loads this
-// library keeps it for the life of the process.
+// B200 (at most one 128 x 256 FP32 partial tile per SM: 18.5 MiB), and every GPU that
+// loads this library keeps it for the life of the process.
 constexpr size_t kStaticScratchBytes = size_t(20) << 20;   // 20 MiB
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
@@ -449,25 +433,20 @@ int fp8_gemm_blockscaled_ws(const uint8_t* A, const float* sA, int64_t ld_sa, co
                             int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
                             void* workspace, size_t workspace_bytes, void* stream) {
   if (M == 0 && N >= 0 && K >= 0) return FP8Q_OK;
-  int st = check_gemm_common(A, B, C, out_dtype, M, N, K, lda, ldb, ldc);
+  int st = check_dense_blockscaled(A, sA, ld_sa, B, sB, ld_sb, b_scale_mode, C, out_dtype, M, N, K,
+                                   lda, ldb, ldc);
   if (st != FP8Q_OK) return st;
-  if (!sA || !sB) return FP8Q_ERR_NULL;
-  if (b_scale_mode != FP8Q_BSCALE_BLOCK128x128 && b_scale_mode != FP8Q_BSCALE_ROW1x128)
-    return FP8Q_ERR_UNSUPPORTED;
-  if (ld_sa < M) return FP8Q_ERR_SHAPE;
-  if (b_scale_mode == FP8Q_BSCALE_ROW1x128 && ld_sb < N) return FP8Q_ERR_SHAPE;
-  if (!aligned(sA, 4) || !aligned(sB, 4)) return FP8Q_ERR_ALIGN;
   if (workspace != nullptr && !aligned(workspace, 16)) return FP8Q_ERR_ALIGN;
   CUtensorMap tmA, tmB;
   if ((st = encode_operand(&tmA, A, K, M, lda, 128)) != FP8Q_OK) return st;
-  if ((st = encode_operand(&tmB, B, K, N, ldb, Cfg1::kBRows)) != FP8Q_OK) return st;
+  if ((st = encode_operand(&tmB, B, K, N, ldb, Cfg1::kBBox)) != FP8Q_OK) return st;
   GemmArgs a{};
   a.sA = sA; a.ld_sa = ld_sa; a.sB = sB; a.ld_sb = ld_sb; a.C = C; a.ldc = ldc;
   a.M = M; a.N = N; a.G = static_cast<int>(K / 128); a.m_offsets = nullptr; a.num_experts = 0;
-  const int64_t tiles = dense_tiles<kPair>(M, N);
+  const int64_t tiles = dense_tiles(M, N);
   if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   const bool row_b = b_scale_mode == FP8Q_BSCALE_ROW1x128, bf16 = out_dtype == FP8Q_OUT_BF16;
-  return dispatch_dense<kPair>(tmA, tmB, a, row_b, bf16, tiles, workspace, workspace_bytes,
+  return dispatch_dense(tmA, tmB, a, row_b, bf16, tiles, workspace, workspace_bytes,
                                static_cast<cudaStream_t>(stream));
 }
 
@@ -547,9 +526,9 @@ int fp8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, size_t* bytes) {
   if (M == 0 || N == 0 || K == 0) return FP8Q_OK;
   if (K % 128 != 0 || N % 128 != 0) return FP8Q_ERR_SHAPE;
   // both B scale modes and output types share the plan
-  const int units = GemmLauncher<kPair, true, false, false, true>::max_units();
+  const int units = GemmLauncher<true, false, false, true>::max_units();
   if (units <= 0) return FP8Q_ERR_CUDA;
-  *bytes = plan_split<kPair>(dense_tiles<kPair>(M, N), K / 128, units).ws_bytes;
+  *bytes = plan_split(dense_tiles(M, N), K / 128, units).ws_bytes;
   return FP8Q_OK;
 }
 
@@ -567,7 +546,7 @@ int fp8_gemm_grouped(const uint8_t* A, const float* sA, int64_t ld_sa, const uin
   if (static_cast<int64_t>(num_groups) * N > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   CUtensorMap tmA, tmB;
   if ((st = encode_operand(&tmA, A, K, max_sum_M, K, 128)) != FP8Q_OK) return st;
-  if ((st = encode_operand(&tmB, W, K, static_cast<uint64_t>(num_groups) * N, K, Cfg1::kBRows)) !=
+  if ((st = encode_operand(&tmB, W, K, static_cast<uint64_t>(num_groups) * N, K, Cfg1::kBBox)) !=
       FP8Q_OK)
     return st;
   GemmArgs a{};
@@ -579,8 +558,8 @@ int fp8_gemm_grouped(const uint8_t* A, const float* sA, int64_t ld_sa, const uin
                         ((N + Cfg1::kN - 1) / Cfg1::kN);
   if (bound > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   const auto s = static_cast<cudaStream_t>(stream);
-  if (out_dtype == FP8Q_OUT_BF16) return run_gemm<kPair, true, false, true, true>(tmA, tmB, a, bound, nullptr, 0, s);
-  return run_gemm<kPair, true, false, true, false>(tmA, tmB, a, bound, nullptr, 0, s);
+  if (out_dtype == FP8Q_OUT_BF16) return run_gemm<true, false, true, true>(tmA, tmB, a, bound, nullptr, 0, s);
+  return run_gemm<true, false, true, false>(tmA, tmB, a, bound, nullptr, 0, s);
 }
 
 int fp8_gemm_nopromo(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB, float* C,
@@ -593,13 +572,13 @@ int fp8_gemm_nopromo(const uint8_t* A, const float* sA, const uint8_t* B, const 
   if (!aligned(sA, 4) || !aligned(sB, 4)) return FP8Q_ERR_ALIGN;
   CUtensorMap tmA, tmB;
   if ((st = encode_operand(&tmA, A, K, M, lda, 128)) != FP8Q_OK) return st;
-  if ((st = encode_operand(&tmB, B, K, N, ldb, fp8q::GemmCfg<false>::kBRows)) != FP8Q_OK) return st;
+  if ((st = encode_operand(&tmB, B, K, N, ldb, Cfg1::kBBox)) != FP8Q_OK) return st;
   GemmArgs a{};
   a.sA = sA; a.ld_sa = 0; a.sB = sB; a.ld_sb = 0; a.C = C; a.ldc = ldc;
   a.M = M; a.N = N; a.G = static_cast<int>(K / 128); a.m_offsets = nullptr; a.num_experts = 0;
-  const int64_t tiles = dense_tiles<false>(M, N);
+  const int64_t tiles = dense_tiles(M, N);
   if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  return run_gemm<false, false, false, false, false>(tmA, tmB, a, tiles, nullptr, 0,
+  return run_gemm<false, false, false, false>(tmA, tmB, a, tiles, nullptr, 0,
                                                      static_cast<cudaStream_t>(stream));
 }
 
@@ -610,14 +589,19 @@ int fp8_gemm_blockscaled_noalloc(const uint8_t* A, const float* sA, int64_t ld_s
                                  int b_scale_mode, void* C, int out_dtype, int64_t M, int64_t N,
                                  int64_t K, int64_t lda, int64_t ldb, int64_t ldc, void* stream) {
   if (M == 0 && N >= 0 && K >= 0) return FP8Q_OK;
-  size_t need = 0;
-  int st = fp8_gemm_workspace_size(M, N, K, &need);
+  // The argument errors are those of fp8_gemm_blockscaled, checked before the plan is sized.
+  int st = check_dense_blockscaled(A, sA, ld_sa, B, sB, ld_sb, b_scale_mode, C, out_dtype, M, N, K,
+                                   lda, ldb, ldc);
   if (st != FP8Q_OK) return st;
+  size_t need = 0;
+  if ((st = fp8_gemm_workspace_size(M, N, K, &need)) != FP8Q_OK) return st;
   if (need > kStaticScratchBytes) return FP8Q_ERR_SHAPE;   // the plan would overflow the array
   void* scratch = static_scratch_address();
   if (scratch == nullptr) return FP8Q_ERR_CUDA;
-  // Nothing in the scratch has to start at zero: every partial tile the reduction reads
-  // is written earlier in the same call.
+  // Nothing in the scratch has to start at zero: in a call that completes, every partial
+  // tile the reduction reads is written earlier in the same call.  After a device-side
+  // timeout (reported by fp8q_get_device_error) a partial may not have been written, and
+  // the reduction then adds a previous call's leftovers: C is undefined in that case.
   return fp8_gemm_blockscaled_ws(A, sA, ld_sa, B, sB, ld_sb, b_scale_mode, C, out_dtype, M, N, K,
                                  lda, ldb, ldc, scratch, kStaticScratchBytes, stream);
 }

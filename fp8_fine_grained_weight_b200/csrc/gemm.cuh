@@ -8,41 +8,41 @@
 // interval of 128 K elements is accumulated on the tensor cores, the partial
 // result is copied out, multiplied by the scaling factors and added into FP32
 // registers.  On Hopper two warpgroups ping-pong so that one promotes while the
-// other issues MMAs (pkd.ac.th webboard 78017 para 4); here the analogue is a
-// double-buffered TMEM accumulator: the tensor core fills buffer g+1 while the
-// epilogue warps drain buffer g.
+// other issues MMAs (pkd.ac.th webboard 78017 para 4); here the analogue is a ring of
+// TMEM accumulator slices: the tensor core fills the next slices while the epilogue
+// warps drain the finished ones.
 //
-// Roles (384-thread CTAs, one per SM, persistent over output tiles):
-//   warp 0      TMA producer: per K-group, the CTA's A tile [128 rows x 128 B] and its
-//               B tile into a shared-memory ring (128-byte swizzle).
-//   warp 1      TMEM owner; in the MMA-issuing CTA also the MMA issuer: 4 x
-//               tcgen05.mma kind::f8f6f4 (K = 32 each) per group into TMEM buffer
-//               (group parity), then tcgen05.commit to free the smem stage and to
-//               publish the partial.
+// Roles (384-thread CTAs, one per SM, persistent over 128 x 256 output tiles):
+//   warp 0      TMA producer: per K-group, the A tile [128 rows x 128 B] and the B tile
+//               [256 rows x 128 B] into a 4-stage shared-memory ring (128-byte swizzle).
+//   warp 1      TMEM owner and MMA issuer: per group 4 x tcgen05.mma kind::f8f6f4 (M128
+//               N256 K32) into a fresh 256-column TMEM accumulator (two, alternating),
+//               then tcgen05.commit to free the smem stage and to publish the partial.
+//               It waits for the stage's operands before the accumulator: the operands
+//               are normally in place long before, while the accumulator comes free just
+//               in time, and the MMAs should follow its release with nothing in between.
 //   warp 2      scale producer: for every group, ahead of the epilogue, copies the
 //               tile's 128 row scales of A and its B scales (2 block scales, or 256
-//               column scales) into an 8-slot shared-memory ring with cp.async.
+//               column scales) into a shared-memory ring with cp.async.  The small copies
+//               queue behind the operand stream in L2, so the ring is deep (24 groups for
+//               block scales, 16 for column scales).
 //   warp 3      idle (it completes the first warpgroup).
-//   warps 4-11  promotion/epilogue: warp w reads TMEM lanes 32*(w%4).., columns
-//               128*((w-4)/4)..; per group: tcgen05.ld -> acc += P * scale in FP32
-//               registers; at tile end: convert and store C.
+//   warps 4-11  promotion/epilogue: warp w reads TMEM lanes 32*(w%4).. and the tile's
+//               columns 128*((w-4)/4)..; per group two 64-column tcgen05.ld and
+//               acc += P * scale in FP32 registers (f32x2 FMAs); the accumulator is freed
+//               after the second load; at the end of the tile: convert and store C.
 //
-// PAIR = true: two CTAs of a cluster share a 256 x 128 output tile with tcgen05
-// cta_group::2.  Each CTA loads its own 128 rows of A and 64 of the 128 rows of B (24 KB
-// per stage, 8 stages), the even CTA issues the M = 256 MMAs and its commits arrive on
-// both CTAs' barriers; each CTA's TMEM holds four 128-column accumulator buffers for its
-// 128 rows and its own epilogue promotes them; the odd CTA frees a buffer with a remote
-// arrive on the even CTA's barrier.  No TMA multicast: every CTA loads its own operands.
-// It passes the parity tests but measures slower than the single-CTA tile (its groups
-// are half as large, so the per-group hand-off is paid twice as often); the launcher
-// does not instantiate it.
-// PAIR = false (used by the promoted GEMMs): one CTA per 128 x 256 tile, B tile of 256
-// rows, 4 stages, two 256-column accumulator buffers; every release is a local arrive.
+// Measured on B200 and not kept (same operands, same parity): a CTA pair with 256 x 256
+// tiles (a third less L2 traffic per FLOP, but the cross-CTA accumulator release slowed
+// every group); MMAs issued as two N = 128 halves into four TMEM slices (more slack per
+// slice, but a single issuing thread then cannot keep the tensor pipe fed); 32-column
+// TMEM loads pipelined with the FMAs, within a group and across groups (the extra
+// registers spill).
 //
 // Registers: the launch gives 168 per thread (3 warps per SM sub-partition).  The
-// first warpgroup gives registers back (setmaxnreg 56) and the two epilogue
-// warpgroups take them (setmaxnreg 224) for the 128-float running sum per thread:
-// 128 * 56 + 256 * 224 = 384 * 168, and per sub-partition 56 + 2 * 224 <= 512.
+// first warpgroup gives registers back (setmaxnreg 40) and the two epilogue
+// warpgroups take them (setmaxnreg 232) for the 128-float running sum per thread:
+// 128 * 40 + 256 * 232 <= 384 * 168, and per sub-partition 40 + 2 * 232 <= 512.
 //
 // PROMOTE = false is the bench-only no-promotion variant: the whole K is
 // accumulated in one TMEM buffer and per-row / per-column (1xK) scales are applied
@@ -59,7 +59,7 @@ constexpr int kBK = 128;
 constexpr int kEpiWarps = 8;
 constexpr int kEpiWarp0 = 4;                      // first epilogue warp (second warpgroup)
 constexpr int kGemmThreads = 32 * (kEpiWarp0 + kEpiWarps);
-constexpr int kRegsCtl = 56, kRegsEpi = 224;      // setmaxnreg split (see above)
+constexpr int kRegsCtl = 40, kRegsEpi = 232;      // setmaxnreg split (see above)
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxGroups = 1024;
 
@@ -86,8 +86,8 @@ struct GemmArgs {
   const int32_t* m_offsets;  // grouped: [E + 1] on the device
   int num_experts;
   // Split-K of the last partial wave (dense only).  Tiles [0, tiles_full) are computed
-  // whole; the remaining tail_tiles are split into tail_split K-chunks, one per CTA of
-  // the last wave, whose FP32 partial tiles go to ws and are summed by
+  // whole; the remaining tail_tiles are split into tail_split K-chunks, one per CTA (or
+  // CTA pair) of the last wave, whose FP32 partial tiles go to ws and are summed by
   // splitk_reduce_kernel.  tail_tiles == 0: no split, ws unused.
   float* ws;
   int tiles_full;
@@ -130,27 +130,25 @@ __device__ __forceinline__ Unit unit_at(int i, const GemmArgs& p, int unit0, int
 
 constexpr uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-template <bool PAIR>
+template <bool ROW_B = false>
 struct GemmCfg {
-  static constexpr int kCG = PAIR ? 2 : 1;              // CTAs per MMA
-  static constexpr int kN = PAIR ? 128 : 256;           // output columns per tile (MMA N)
-  static constexpr int kAccBufs = kTmemCols / kN;       // TMEM accumulator buffers
-  static constexpr int kSetCols = kN / 2;               // columns per epilogue column set
-  static constexpr int kStages = PAIR ? 8 : 4;
-  static constexpr int kTileM = 128 * kCG;              // output rows per (pair) tile
-  static constexpr int kBRows = kN / kCG;               // rows of B each CTA loads
-  static constexpr uint32_t kABytes = 128 * kBK;        // per CTA per stage
-  static constexpr uint32_t kBBytes = kBRows * kBK;
-  static constexpr uint32_t kStageTx = (kABytes + kBBytes) * kCG;  // bytes per full barrier phase
-  // accumulator release: every epilogue thread arrives (1 CTA); one remote arrive per
-  // epilogue warp of both CTAs (pair)
-  static constexpr uint32_t kTemptyArrivals = PAIR ? kCG * kEpiWarps : 32 * kEpiWarps;
+  static constexpr int kN = 256;                        // output columns per tile (MMA N)
+  static constexpr int kTileM = 128;                    // output rows per tile (MMA M)
+  static constexpr int kAccBufs = kTmemCols / kN;       // TMEM accumulators (groups in flight)
+  static constexpr int kSetCols = kN / 2;               // columns per epilogue warpgroup
+  static constexpr int kStages = 4;
+  static constexpr int kBBox = kN;                      // B rows per TMA box
+  static constexpr uint32_t kABytes = 128 * kBK;        // per stage
+  static constexpr uint32_t kBBytes = kN * kBK;
+  static constexpr uint32_t kStageTx = kABytes + kBBytes;  // bytes per full barrier phase
   // shared memory, byte offsets from the 1024-aligned base
   static constexpr uint32_t a = 0;
   static constexpr uint32_t b = a + kStages * kABytes;
   static constexpr uint32_t bars = b + kStages * kBBytes;
-  static constexpr int kScaleSlots = 8;                  // scale ring depth (groups)
-  static constexpr uint32_t kSlotFloats = 128 + kN;      // A row scales + B scales
+  // Scale ring: a slot holds one group's 128 A row scales and its B scales (the tile's
+  // kN column scales in ROW mode; its kN / 128 block scales, padded to 4, otherwise).
+  static constexpr int kScaleSlots = ROW_B ? 16 : 24;
+  static constexpr uint32_t kSlotFloats = 128 + (ROW_B ? kN : 4);
   // full[S], empty[S], tfull[NB], tempty[NB], drain, sfull[R], sempty[R]
   static constexpr uint32_t n_bars = 2 * kStages + 2 * kAccBufs + 1 + 2 * kScaleSlots;
   static constexpr uint32_t misc = align_up(bars + 8 * n_bars, 16);   // tmem slot, abort flag
@@ -161,9 +159,10 @@ struct GemmCfg {
   static constexpr uint32_t smem_bytes = end + 1024;                  // + base alignment slack
   static_assert(a % 1024 == 0 && b % 1024 == 0 && kABytes % 1024 == 0 && kBBytes % 1024 == 0,
                 "swizzle atoms");
-  static_assert(sbrow % 16 == 0 && sring % 16 == 0 && kSlotFloats % 4 == 0,
+  static_assert(sbrow % 16 == 0 && sring % 16 == 0 && kSlotFloats % 4 == 0 && kN / 128 <= 4,
                 "float4 reads of the scale slots");
-  static_assert(kSetCols % 64 == 0 && kN % 128 == 0, "epilogue column sets of 64-column loads");
+  static_assert(kSetCols % 64 == 0 && kAccBufs >= 2, "64-column loads; two accumulators");
+  static_assert(kN % 16 == 0 && kN <= 256 && kBBox <= 256, "MMA N and TMA box");
   static_assert(smem_bytes <= 232448, "fits the 227 KB opt-in shared memory");
 };
 
@@ -224,17 +223,38 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-template <bool PAIR, bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16>
+// Promotion of one 32-column chunk of a slice into this thread's running sums:
+// acc[j] += P * s (BLOCK: one scale for the whole chunk) or acc[j] += (P * sB[n]) * sA
+// (ROW: a scale per column, read from shared memory as float4).
+template <bool ROW_B>
+__device__ __forceinline__ void promote_chunk(float2* acc, const uint32_t* r, float2 sc2,
+                                              float2 sa2, const float* sbv) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) {
+    const float2 p0 = make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
+    const float2 p1 = make_float2(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+    float2& a0 = acc[j / 2];
+    float2& a1 = acc[j / 2 + 1];
+    if (ROW_B) {
+      const float4 b4 = *reinterpret_cast<const float4*>(sbv + j);
+      a0 = __ffma2_rn(__fmul2_rn(p0, make_float2(b4.x, b4.y)), sa2, a0);
+      a1 = __ffma2_rn(__fmul2_rn(p1, make_float2(b4.z, b4.w)), sa2, a1);
+    } else {
+      a0 = __ffma2_rn(p0, sc2, a0);
+      a1 = __ffma2_rn(p1, sc2, a1);
+    }
+  }
+}
+
+template <bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_fp8_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA,
                                 const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
-  using Cfg = GemmCfg<PAIR>;
-  constexpr int CG = Cfg::kCG;
+  using Cfg = GemmCfg<ROW_B>;
   constexpr int S = Cfg::kStages;
   constexpr int NB = Cfg::kAccBufs;
   constexpr int kN = Cfg::kN;
   constexpr int kSetCols = Cfg::kSetCols;
-  static_assert(PROMOTE || !PAIR, "the no-promotion variant runs on single CTAs");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -256,9 +276,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.G;
-  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;   // CTA 0 of a pair issues the MMAs
-  const bool mma_cta = rank == 0;
-  const int unit0 = blockIdx.x / CG, units = gridDim.x / CG;   // cluster index / count
+  const int unit0 = blockIdx.x, units = gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -267,7 +285,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < NB; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), Cfg::kTemptyArrivals);
+      mbar_init(tempty_bar(b), 32 * kEpiWarps);   // every epilogue thread frees it
     }
     mbar_init(drain_bar, 1);
     for (int r = 0; r < R; ++r) {
@@ -282,8 +300,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc<CG>(smem_u32(tmem_slot), kTmemCols);
-    tmem_relinquish<CG>();
+    tmem_alloc<1>(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish<1>();
   }
 
   const int nt_total = static_cast<int>((p.N + kN - 1) / kN);
@@ -307,7 +325,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (PAIR) cluster_sync();       // the peer's barriers are initialised before any remote use
   tc_fence_after();
   if (GROUPED) num_tiles = sched[p.num_experts];
   const int n_units = units_of(p, num_tiles, unit0, units);
@@ -322,39 +339,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         bool ok = true;
         for (int ui = 0; ok && ui < n_units; ++ui) {
           const Unit u = unit_at(ui, p, unit0, units, G);
-          const Tile tl = decode_tile<GROUPED, Cfg::kTileM, Cfg::kN>(u.tile, p, mt_total, nt_total, sched);
-          const int32_t arow = static_cast<int32_t>(tl.row0 + 128 * rank);
-          const int32_t brow = static_cast<int32_t>(tl.brow0 + Cfg::kBRows * rank);
+          const Tile tl = decode_tile<GROUPED, Cfg::kTileM, kN>(u.tile, p, mt_total, nt_total, sched);
           for (int g = u.g0; g < u.g1; ++g, ++it) {
             const int s = it % S;
-            const uint32_t ph = (it / S) & 1u;
-            if (!mbar_wait(empty_bar(s), ph ^ 1u, kSiteProducer, abort_flag)) { ok = false; break; }
-            if (mma_cta) mbar_arrive_expect_tx(full_bar(s), Cfg::kStageTx);
-            const uint32_t dst_a = sbase + Cfg::a + s * Cfg::kABytes;
-            const uint32_t dst_b = sbase + Cfg::b + s * Cfg::kBBytes;
-            if (PAIR) {
-              const uint32_t fb = map_shared_rank(full_bar(s), 0);   // the MMA CTA's barrier
-              tma_load_2d_pair(dst_a, &tmA, fb, g * kBK, arow);
-              tma_load_2d_pair(dst_b, &tmB, fb, g * kBK, brow);
-            } else {
-              tma_load_2d(dst_a, &tmA, full_bar(s), g * kBK, arow);
-              tma_load_2d(dst_b, &tmB, full_bar(s), g * kBK, brow);
-            }
+            if (!mbar_wait(empty_bar(s), ((it / S) & 1u) ^ 1u, kSiteProducer, abort_flag)) { ok = false; break; }
+            mbar_arrive_expect_tx(full_bar(s), Cfg::kStageTx);
+            tma_load_2d(sbase + Cfg::a + s * Cfg::kABytes, &tmA, full_bar(s), g * kBK,
+                        static_cast<int32_t>(tl.row0));
+            tma_load_2d(sbase + Cfg::b + s * Cfg::kBBytes, &tmB, full_bar(s), g * kBK,
+                        static_cast<int32_t>(tl.brow0));
           }
         }
-        // Every issued load lands before the CTA can exit.  The MMA CTA watches its full
-        // barriers (bounded; loads finish on their own).  The other CTA's loads complete on
-        // the MMA CTA's barriers; in the normal path they were all consumed before the
-        // final cluster barrier, after an abort the teardown below waits a fixed while.
-        if (mma_cta) {
-          const uint32_t first = it > static_cast<uint32_t>(S) ? it - S : 0;
-          for (uint32_t j = first; j < it; ++j)
-            mbar_wait(full_bar(j % S), (j / S) & 1u, kSiteDrain, nullptr);
-        }
+        // every issued load lands before the CTA can exit (bounded; loads end on their own)
+        const uint32_t first = it > static_cast<uint32_t>(S) ? it - S : 0;
+        for (uint32_t j = first; j < it; ++j)
+          mbar_wait(full_bar(j % S), (j / S) & 1u, kSiteDrain, nullptr);
       }
     } else if (warp == 1) {
       // ---------------------------------------------------------- MMA issuer
-      if (lane == 0 && mma_cta) {
+      if (lane == 0) {
         constexpr uint32_t idesc = idesc_e4m3_f32(Cfg::kTileM, kN);
         uint32_t it = 0, acc_it = 0;
         bool ok = true;
@@ -362,17 +365,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const Unit u = unit_at(ui, p, unit0, units, G);
           uint32_t buf = 0;
           for (int g = u.g0; g < u.g1; ++g, ++it) {
-            if (PROMOTE || g == u.g0) {
+            const bool fresh = PROMOTE || g == u.g0;   // a new accumulator for this group
+            const bool publish = PROMOTE || g == u.g1 - 1;
+            const int s = it % S;
+            // The stage's operands first (normally long in place), then the accumulator,
+            // which comes free just in time: nothing should separate its release from
+            // the MMAs.
+            if (!mbar_wait(full_bar(s), (it / S) & 1u, kSiteMmaFull, abort_flag)) {
+              ok = false;
+              break;
+            }
+            if (fresh) {
               buf = acc_it % NB;
               if (!mbar_wait(tempty_bar(buf), ((acc_it / NB) & 1u) ^ 1u, kSiteMmaEmpty, abort_flag)) {
                 ok = false;
                 break;
               }
-            }
-            const int s = it % S;
-            if (!mbar_wait(full_bar(s), (it / S) & 1u, kSiteMmaFull, abort_flag)) {
-              ok = false;
-              break;
             }
             tc_fence_after();
             const uint32_t d = tmem_base + buf * kN;
@@ -381,31 +389,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < kBK / 32; ++kk) {
               const uint32_t accumulate = PROMOTE ? (kk > 0) : (g > u.g0 || kk > 0);
-              mma_f8<CG>(d, smem_desc_k_sw128(a_addr + 32 * kk), smem_desc_k_sw128(b_addr + 32 * kk),
-                         idesc, accumulate);
+              mma_f8<1>(d, smem_desc_k_sw128(a_addr + 32 * kk), smem_desc_k_sw128(b_addr + 32 * kk),
+                        idesc, accumulate);
             }
-            if (PAIR) mma_commit_pair(empty_bar(s), 0x3); else mma_commit<1>(empty_bar(s));
-            if (PROMOTE || g == u.g1 - 1) {
-              if (PAIR) mma_commit_pair(tfull_bar(buf), 0x3); else mma_commit<1>(tfull_bar(buf));
+            mma_commit<1>(empty_bar(s));
+            if (publish) {
+              mma_commit<1>(tfull_bar(buf));
               ++acc_it;
             }
           }
         }
         // All MMAs this thread issued complete before TMEM is released.
-        mma_commit<CG>(drain_bar);
+        mma_commit<1>(drain_bar);
         mbar_wait(drain_bar, 0, kSiteDrain, nullptr);
       }
     } else if (warp == 2 && PROMOTE) {
       // ---------------------------------------------------------- scale producer
-      // Slot layout: [0, 128) A scales of this CTA's 128 rows; [128, 128 + kN) B scales:
-      // the tile's kN column scales (ROW mode) or, for 128x128 weight blocks, the kN / 128
+      // Slot layout: [0, 128) A scales of the tile's 128 rows; then the B scales: the
+      // tile's kN column scales (ROW mode) or, for 128x128 weight blocks, the kN / 128
       // blocks' scales.
       uint32_t it = 0;
       bool ok = true;
       for (int ui = 0; ok && ui < n_units; ++ui) {
         const Unit u = unit_at(ui, p, unit0, units, G);
-        const Tile tl = decode_tile<GROUPED, Cfg::kTileM, Cfg::kN>(u.tile, p, mt_total, nt_total, sched);
-        const int64_t r0 = tl.row0 + 128 * rank;
+        const Tile tl = decode_tile<GROUPED, Cfg::kTileM, kN>(u.tile, p, mt_total, nt_total, sched);
         const float* sB_tile =
             ROW_B ? nullptr : p.sB + (static_cast<int64_t>(tl.expert) * (p.N / 128) + tl.col0 / 128) * G;
         for (int g = u.g0; g < u.g1; ++g, ++it) {
@@ -418,7 +425,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const float* sa_g = p.sA + static_cast<int64_t>(g) * p.ld_sa;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const int64_t m = r0 + 32 * j + lane;
+            const int64_t m = tl.row0 + 32 * j + lane;
             cp_async_4(slot + 4u * (32 * j + lane), sa_g + (m < tl.row_end ? m : 0), m < tl.row_end);
           }
           if (ROW_B) {
@@ -443,33 +450,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int ew = warp - kEpiWarp0;
     const int quad = warp & 3;              // TMEM lanes this warp may access
     const int set = ew >> 2;                // column half of the tile
-    const int row_in_tile = static_cast<int>(128 * rank) + quad * 32 + lane;
+    const int row_in_tile = quad * 32 + lane;
     const int tid_in_set = (ew & 3) * 32 + lane;
     float* sb_slots = sbrow + set * 2 * 128;
-    // Release of an accumulator buffer: each thread arrives on its own CTA's barrier; in
-    // a pair, one arrive per warp on the MMA CTA's barrier.
-    auto release = [&](uint32_t buf) {
+    auto release = [&](uint32_t buf) {      // every epilogue thread arrives
       tc_fence_before();
-      if (PAIR) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(map_shared_rank(tempty_bar(buf), 0));
-      } else {
-        mbar_arrive(tempty_bar(buf));
-      }
+      mbar_arrive(tempty_bar(buf));
     };
     // The epilogue never leaves its loops early: after an abort it keeps walking the
     // (uniform) tile/group structure without touching TMEM, so that every thread of a
     // column set reaches the same named barriers.
-    constexpr int kLoads = kSetCols / 64;   // 64-column TMEM loads per group
     uint32_t acc_it = 0;
     bool ok = true;
+    uint32_t rbuf[64];                      // one 64-column TMEM load
     for (int ui = 0; ui < n_units; ++ui) {
       const Unit u = unit_at(ui, p, unit0, units, G);
-      const Tile tl = decode_tile<GROUPED, Cfg::kTileM, Cfg::kN>(u.tile, p, mt_total, nt_total, sched);
-      const int64_t m = tl.row0 + row_in_tile;
-      const bool row_ok = m < tl.row_end;
-      const int64_t n0 = tl.col0 + set * kSetCols;
-      const bool cols_ok = n0 < p.N;
+      bool warp_idle;
+      {
+        // warp-uniform: none of this warp's 32 rows is inside the tile's rows (an expert's
+        // short last row tile), so its partials are never read.  (The tile is decoded
+        // again for the stores, so that nothing of it stays live through the group loop.)
+        const Tile tl = decode_tile<GROUPED, Cfg::kTileM, kN>(u.tile, p, mt_total, nt_total, sched);
+        warp_idle = tl.row0 + row_in_tile - lane >= tl.row_end;
+      }
       // acc[i] holds columns 2i, 2i+1 of this thread's row (packed FP32 pairs: the
       // promotion runs on the f32x2 FMA path, two accumulations per instruction).
       float2 acc[kSetCols / 2];
@@ -481,47 +484,41 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           // This group's scales, staged by the scale producer (the ring advances with
           // every group of every tile, in the same order as acc_it).
           const int r = acc_it % R;
-          const float* slot = sring + Cfg::kSlotFloats * r;
+          const int slot = Cfg::kSlotFloats * r;
           if (ok) ok = mbar_wait(sfull_bar(r), (acc_it / R) & 1u, kSiteScales, abort_flag);
-          const float sa_cur = slot[quad * 32 + lane];
-          const float sb_cur = ROW_B ? 0.0f : slot[128 + set * kSetCols / 128];
-          const float* sbv = slot + 128 + set * kSetCols;   // ROW mode column scales
+          const float sa_cur = sring[slot + quad * 32 + lane];
+          const float sb_cur = ROW_B ? 0.0f : sring[slot + 128 + set * kSetCols / 128];
+          const int sb = slot + 128 + set * kSetCols;        // ROW mode column scales
           const uint32_t buf = acc_it % NB;
           if (ok) ok = mbar_wait(tfull_bar(buf), (acc_it / NB) & 1u, kSiteEpilogue, abort_flag);
-          if (ok) {
+          ok = __all_sync(0xFFFFFFFFu, ok);  // warp-uniform: TMEM loads are per warp
+          if (ok && !warp_idle) {
             tc_fence_after();
             const uint32_t taddr =
                 tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + buf * kN + set * kSetCols;
             const float2 sc2 = make_float2(sa_cur * sb_cur, sa_cur * sb_cur);
             const float2 sa2 = make_float2(sa_cur, sa_cur);
 #pragma unroll
-            for (int h = 0; h < kLoads; ++h) {
-              uint32_t r[64];
-              tmem_ld_64cols(taddr + h * 64, r);
-              tmem_ld_wait();
-              if (h == kLoads - 1) release(buf);   // TMEM buffer free for group g + NB
-#pragma unroll
-              for (int j = 0; j < 64; j += 4) {
-                const float2 p0 = make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
-                const float2 p1 = make_float2(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
-                float2& a0 = acc[(h * 64 + j) / 2];
-                float2& a1 = acc[(h * 64 + j) / 2 + 1];
-                if (ROW_B) {
-                  const float4 b4 = *reinterpret_cast<const float4*>(sbv + h * 64 + j);
-                  a0 = __ffma2_rn(__fmul2_rn(p0, make_float2(b4.x, b4.y)), sa2, a0);
-                  a1 = __ffma2_rn(__fmul2_rn(p1, make_float2(b4.z, b4.w)), sa2, a1);
-                } else {
-                  a0 = __ffma2_rn(p0, sc2, a0);
-                  a1 = __ffma2_rn(p1, sc2, a1);
-                }
-              }
+            for (int h = 0; h < kSetCols / 64; ++h) {
+              tmem_ld_64cols(taddr + h * 64, rbuf);
+              tmem_ld_wait_regs(rbuf);
+              if (h == kSetCols / 64 - 1) release(buf);   // TMEM buffer free for group g + NB
+              promote_chunk<ROW_B>(acc + 32 * h, rbuf, sc2, sa2, sring + sb + 64 * h);
+              promote_chunk<ROW_B>(acc + 32 * h + 16, rbuf + 32, sc2, sa2, sring + sb + 64 * h + 32);
             }
+          } else if (ok) {
+            release(buf);
           }
           mbar_arrive(sempty_bar(r));   // scales of this group consumed
           ++acc_it;
         }
       } else {
         // no promotion: one accumulator over all of K, scaled once by sA[m] * sB[n]
+        const Tile tl = decode_tile<GROUPED, Cfg::kTileM, kN>(u.tile, p, mt_total, nt_total, sched);
+        const int64_t m = tl.row0 + row_in_tile;
+        const bool row_ok = m < tl.row_end;
+        const int64_t n0 = tl.col0 + set * kSetCols;
+        const bool cols_ok = n0 < p.N;
         const float sa = row_ok ? __ldg(p.sA + m) : 0.0f;
         float* slot = sb_slots;
         named_bar_sync(1 + set, 128);   // previous tile's readers are done with the slot
@@ -530,20 +527,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         named_bar_sync(1 + set, 128);
         const uint32_t buf = acc_it % NB;
         if (ok) ok = mbar_wait(tfull_bar(buf), (acc_it / NB) & 1u, kSiteEpilogue, abort_flag);
+        ok = __all_sync(0xFFFFFFFFu, ok);
         if (ok) {
           tc_fence_after();
           const uint32_t taddr =
               tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + buf * kN + set * kSetCols;
           const float2 sa2 = make_float2(sa, sa);
 #pragma unroll
-          for (int h = 0; h < kLoads; ++h) {
-            uint32_t r[64];
-            tmem_ld_64cols(taddr + h * 64, r);
-            tmem_ld_wait();
-            if (h == kLoads - 1) release(buf);
+          for (int h = 0; h < kSetCols / 64; ++h) {
+            tmem_ld_64cols(taddr + h * 64, rbuf);
+            tmem_ld_wait_regs(rbuf);
+            if (h == kSetCols / 64 - 1) release(buf);
 #pragma unroll
             for (int j = 0; j < 64; j += 2) {
-              const float2 pr = make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
+              const float2 pr = make_float2(__uint_as_float(rbuf[j]), __uint_as_float(rbuf[j + 1]));
               const float2 sb2 = *reinterpret_cast<const float2*>(slot + h * 64 + j);
               acc[(h * 64 + j) / 2] = __fmul2_rn(__fmul2_rn(pr, sa2), sb2);
             }
@@ -553,6 +550,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
 
       // ---- store the tile's rows: this thread owns row m, columns n0 .. n0 + kSetCols
+      const Tile tl = decode_tile<GROUPED, Cfg::kTileM, kN>(u.tile, p, mt_total, nt_total, sched);
+      const int64_t m = tl.row0 + row_in_tile;
+      const bool row_ok = m < tl.row_end;
+      const int64_t n0 = tl.col0 + set * kSetCols;
+      const bool cols_ok = n0 < p.N;
       if (ok && u.ws_index >= 0) {
         // split-K partial: the whole tile row (zeros outside C), summed later in fixed order
         float* wrow = p.ws + (static_cast<int64_t>(u.ws_index) * Cfg::kTileM + row_in_tile) * kN +
@@ -591,25 +593,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
-  if (PAIR) {
-    // After an abort the other CTA's in-flight loads into this CTA's shared memory are
-    // not tracked by any local barrier: give them a fixed, generous time to land.
-    if (*abort_flag) {
-      const uint64_t t0 = globaltimer();
-      while (globaltimer() - t0 < 200000ull) {
-      }
-    }
-    __syncwarp();
-    cluster_sync();
-  }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc<CG>(tmem_base, kTmemCols);
-  }
-  if (PAIR) {
-    __syncwarp();
-    cluster_sync();               // neither CTA exits while its peer may still address it
+    tmem_dealloc<1>(tmem_base, kTmemCols);
   }
 }
 

@@ -228,9 +228,12 @@ int fp8_gemm_blockscaled_ws(const uint8_t* A, const float* sA, int64_t ld_sa, co
  *    stream capture.
  *  - Returns FP8Q_ERR_SHAPE when the problem's split would need more than 20 MiB
  *    (possible only on a GPU with more SMs), besides the errors of fp8_gemm_blockscaled.
+ *  - Argument errors are those of fp8_gemm_blockscaled and are checked first.
  *  - All calls share the one array, which keeps the previous call's contents (nothing in
  *    it needs to start at zero).  Calls that can overlap on the GPU -- on different
  *    streams, or from different threads -- race on it and must be serialized by the caller.
+ *  - If fp8q_get_device_error then reports a timeout, C is undefined (the reduction may
+ *    have added partial tiles left by an earlier call).
  */
 int fp8_gemm_blockscaled_noalloc(const uint8_t* A, const float* sA, int64_t ld_sa,
                                  const uint8_t* B, const float* sB, int64_t ld_sb,

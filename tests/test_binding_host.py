@@ -2,6 +2,8 @@
 the arguments it hands to the C ABI.  The library call is recorded instead of made and
 the CUDA-tensor requirement is lifted, so CPU tensors stand in for device buffers; the
 shapes are the ones the GPU tests, the bench and the FP8 linear layer use."""
+import collections
+
 import pytest
 import torch
 
@@ -162,7 +164,7 @@ def test_split_workspace_is_per_stream(calls, monkeypatch):
     """The cached split-K workspace is keyed by (device, stream): GEMMs on one stream share
     it (they run in order), GEMMs on different streams never do."""
     monkeypatch.setattr(fq, "workspace_bytes", lambda M, N, K: 4096)
-    monkeypatch.setattr(fq, "_WORKSPACE", {})
+    monkeypatch.setattr(fq, "_WORKSPACE", collections.OrderedDict())
     qa, sa, qb, sb = E(256, 384), E(3, 256, dtype=f32), E(512, 384), E(4, 3, dtype=f32)
     ptrs = []
     for stream in (11, 11, 22):
@@ -176,3 +178,25 @@ def test_split_workspace_is_per_stream(calls, monkeypatch):
     fq.gemm_blockscaled(qa, sa, qb, sb, workspace=own)       # a caller's buffer is used as is
     assert calls[-1][1][-3] == own.data_ptr()
 
+
+
+def test_split_workspace_cache_is_bounded(calls, monkeypatch):
+    """At most _WORKSPACE_MAX per-stream buffers are cached; the least recently used one is
+    dropped first, and a stream that comes back gets a fresh buffer."""
+    monkeypatch.setattr(fq, "workspace_bytes", lambda M, N, K: 4096)
+    monkeypatch.setattr(fq, "_WORKSPACE", collections.OrderedDict())
+    monkeypatch.setattr(fq, "_WORKSPACE_MAX", 3)
+    qa, sa, qb, sb = E(256, 384), E(3, 256, dtype=f32), E(512, 384), E(4, 3, dtype=f32)
+
+    def on(stream):
+        monkeypatch.setattr(fq, "_stream", lambda t, s=stream: s)
+        fq.gemm_blockscaled(qa, sa, qb, sb)
+        return calls[-1][1][-3]
+
+    first = on(1)
+    for stream in (2, 3, 1, 4):            # stream 1 is used again, so 2 is the oldest
+        on(stream)
+    assert [k[1] for k in fq._WORKSPACE] == [3, 1, 4]
+    assert on(1) == first                  # still cached
+    on(2)                                  # evicted earlier: a new buffer, 3 drops out
+    assert [k[1] for k in fq._WORKSPACE] == [4, 1, 2]
