@@ -318,6 +318,8 @@ def run_gpu(args, rank, world):
         res["accumulation_study"] = accumulation_study(fq)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w, a_bits, b_bits, budget_s=args.cpu_budget)
+        if not args.no_configs:
+            res["cpu_baseline_configs"] = cpu_baseline_configs()
     return res
 
 
@@ -667,63 +669,126 @@ def spot_check(w, qA, sA, qB, sB, C, b_rowwise: bool = False):
 
 # ------------------------------------------------------------------------------ CPU oracle
 
-def cpu_baseline(w, a_bits, b_bits, budget_s: float = 20.0):
-    """The oracle, as it stands, on the host cores: W quantized in full once, then A rows in
-    chunks (1x128 quantization + FP64 dequantize + dgemm) until the budget is spent; the
-    per-step time is extrapolated to all M rows."""
-    import oracle
-    cores = os.cpu_count()
-    t0 = time.perf_counter()
-    qb, sb = oracle.quant_weight_128x128(b_bits, w.pow2_b)
-    Bd = oracle.dequant_blocks(qb, sb)
-    t_w = time.perf_counter() - t0
-    rows_done, t_rows, chunk = 0, 0.0, 64
-    while t_rows < budget_s and rows_done < w.M:
+class OracleSample:
+    """The oracle on a sample of a workload, one component at a time, each time scaled to the
+    whole workload by its share of the work (the oracle's work is linear in each):
+
+      A quantization (1x128 tiles) of `a_rows` rows      x  (total A rows) / a_rows
+      W quantization (128x128 blocks) of `w_rows` rows   x  (total W rows) / w_rows
+      FP64 dequantize + dgemm of `a_rows` rows by one
+        expert's full W                                  x  (GEMM FLOPs) / (sample FLOPs)
+
+    The dequantized W of the GEMM leg is prepared once, outside the timed components.  W
+    rows are taken in turn (a different 128-row-aligned slice each call).  Used by both the
+    `cpu_baseline` leg and the reference arm, so that the two CPU figures measure the same."""
+
+    def __init__(self, w, a_bits, b_bits, a_rows=64, w_rows=1024):
+        import oracle
+        self.oracle, self.w = oracle, w
+        self.a_rows = min(a_rows, a_bits.shape[0])
+        wb = b_bits if b_bits.ndim == 2 else b_bits[0]           # one expert's weights
+        self.w_rows = min(w_rows, wb.shape[0])
+        self.a_bits, self.wb = a_bits, wb
+        if w.b_rowwise:
+            qb, sb = oracle.quant_act_1x128(wb, w.pow2_b)
+            self.Bd = oracle.dequant_rows_groupmajor(qb, sb)
+        else:
+            qb, sb = oracle.quant_weight_128x128(wb, w.pow2_b)
+            self.Bd = oracle.dequant_blocks(qb, sb)
+        self.w_rows_total = w.N * max(1, w.experts)
+        self._next = 0
+
+    def step(self) -> float:
+        """Seconds the oracle takes for the whole workload, extrapolated from one sample."""
+        o, w = self.oracle, self.w
+        r0 = (self._next * self.a_rows) % max(1, self.a_bits.shape[0] - self.a_rows + 1)
+        a = self.a_bits[r0:r0 + self.a_rows]
+        w0 = (self._next * self.w_rows) % max(1, self.wb.shape[0] - self.w_rows + 1) // 128 * 128
+        wslice = self.wb[w0:w0 + self.w_rows]
+        self._next += 1
+        t0 = time.perf_counter()
+        qa, sa = o.quant_act_1x128(a, w.pow2_a)
         t1 = time.perf_counter()
-        r = slice(rows_done, min(w.M, rows_done + chunk))
-        qa, sa = oracle.quant_act_1x128(a_bits[r], w.pow2_a)
-        Ad = oracle.dequant_rows_groupmajor(qa, sa)
-        _ = Ad @ Bd.T
-        t_rows += time.perf_counter() - t1
-        rows_done = r.stop
-    t_step = t_w + t_rows * (w.M / rows_done)
+        if w.b_rowwise:
+            o.quant_act_1x128(wslice, w.pow2_b)
+        else:
+            o.quant_weight_128x128(wslice, w.pow2_b)
+        t2 = time.perf_counter()
+        Ad = o.dequant_rows_groupmajor(qa, sa)
+        _ = Ad @ self.Bd.T
+        t3 = time.perf_counter()
+        sample_flops = 2.0 * self.a_rows * self.Bd.shape[0] * w.K
+        return ((t1 - t0) * w.M / self.a_rows + (t2 - t1) * self.w_rows_total / self.w_rows
+                + (t3 - t2) * w.gemm_flops / sample_flops)
+
+    def describe(self) -> str:
+        return (f"per sample: 1x128 quantization of {self.a_rows} A rows, "
+                f"{'1x128' if self.w.b_rowwise else '128x128'} quantization of {self.w_rows} W rows, "
+                f"FP64 dequantize + dgemm of {self.a_rows} rows x [{self.Bd.shape[0]}, {self.w.K}]; "
+                f"each scaled to the whole workload by its share of the work")
+
+
+def cpu_baseline(w, a_bits, b_bits, budget_s: float = 15.0):
+    """The oracle, as it stands, on the host cores: samples of the workload (OracleSample)
+    until the budget is spent; the median extrapolated step time gives the metric."""
+    cores = os.cpu_count()
+    smp = OracleSample(w, a_bits, b_bits)
+    times, t_end = [], time.perf_counter() + budget_s
+    while time.perf_counter() < t_end or len(times) < 3:
+        times.append(smp.step())
+    t_step = statistics.median(times)
     return {"value": round(w.gemm_flops / t_step / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
-            "kind": "oracle",
-            "sample": f"full W quantization ({t_w:.2f} s) + {rows_done} of {w.M} A rows "
-                      f"(quantize, FP64 dequantize, dgemm: {t_rows:.2f} s), per-step time "
-                      f"extrapolated to all rows; numpy BLAS and OpenMP threads = host cores"}
+            "kind": "oracle", "samples": len(times),
+            "sample": smp.describe() + f"; median over {len(times)} samples; numpy BLAS and "
+                                       f"OpenMP threads = host cores"}
+
+
+def cpu_baseline_configs(budget_s: float = 4.0) -> dict:
+    """The oracle per workload (prefill and decode per expert, wgrad), a few seconds each, on
+    the workloads' own seeded inputs (the first rows of A; one expert's weights)."""
+    out = {}
+    for name in ("prefill", "decode", "wgrad"):
+        w = workloads.ALL[name]()
+        rng = workloads.rng_for(3 if name == "prefill" else (4 if name == "decode" else 5), 7)
+        a_bits = workloads.normal_bf16(rng, (256, w.K), w.a_std, w.a_outliers)
+        b_bits = workloads.normal_bf16(rng, (w.N, w.K), w.b_std)
+        smp = OracleSample(w, a_bits, b_bits, a_rows=64, w_rows=min(1024, w.N))
+        times, t_end = [], time.perf_counter() + budget_s
+        while time.perf_counter() < t_end or len(times) < 2:
+            times.append(smp.step())
+        t = statistics.median(times)
+        out[name] = {"workload": w.name, "value": round(w.gemm_flops / t / 1e12, 6), "unit": "TFLOP/s",
+                     "seconds_per_pass": round(t, 3), "samples": len(times),
+                     "sample": smp.describe() + (f"; weights of one expert, W quantization scaled "
+                                                 f"to all {w.experts} experts" if w.experts else "")}
+    return out
 
 
 def run_reference(args):
-    """Reference arm: the CPU oracle on a bounded sample per step (8 rows x 128 columns)."""
-    import oracle
+    """Reference arm: the CPU oracle (this project's reference: the pages hold no code) on the
+    dense workload, one OracleSample per step, with the same sampling as `cpu_baseline`;
+    the step time is the median of the steps' extrapolated times."""
     w = workloads.ALL[args.workload]()
-    rng = np.random.default_rng(0)
-    a_bits = workloads.normal_bf16(rng, (8, w.K), w.a_std, w.a_outliers)
-    b_bits = workloads.normal_bf16(rng, (128, w.K), w.b_std)
-    flops = 2.0 * 8 * 128 * w.K
-
-    def step():
-        qa, sa = oracle.quant_act_1x128(a_bits, w.pow2_a)
-        qb, sb = oracle.quant_weight_128x128(b_bits, w.pow2_b)
-        oracle.gemm_blockscaled_ref(qa, sa, qb, sb)
-
+    rows = min(w.M, 256)
+    a_bits = w.gen_a()[:rows] if w.M <= 4096 else workloads.normal_bf16(
+        np.random.default_rng(0), (rows, w.K), w.a_std, w.a_outliers)
+    b_bits = w.gen_b()
+    smp = OracleSample(w, a_bits, b_bits)
     for _ in range(max(args.warmup, 3)):
-        step()
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        step()
-    dt = (time.perf_counter() - t0) / args.steps
-    v = round(flops / dt / 1e12, 6)
+        smp.step()
+    t_wall0 = time.perf_counter()
+    times = [smp.step() for _ in range(args.steps)]
+    wall = time.perf_counter() - t_wall0
+    t_step = statistics.median(times)
+    v = round(w.gemm_flops / t_step / 1e12, 6)
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": 1,
-            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(dt * 1e3, 4),
+            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(t_step * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64 (oracle)", "data": "synthetic",
             "config": bench_config(w, 1),
-            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": os.cpu_count(),
-                             "kind": "oracle",
-                             "sample": f"per step: 8 rows x 128 columns x K={w.K} of the workload "
-                                       f"(1x128 + 128x128 quantization, FP64 GEMM)"},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                             "sample": smp.describe() + f"; {args.steps} samples in {wall:.1f} s of "
+                                                        f"wall time, median extrapolated step"},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
