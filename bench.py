@@ -351,8 +351,10 @@ def _time_ms(fn, reps, flush_l2, warmup=2):
     return tot / reps
 
 
-def _dev_normal(shape, std, seed):
-    """Seeded normal bf16 samples generated on the device (timing-only inputs)."""
+def _dev_normal(shape, std, seed, outlier_frac=0.0):
+    """Seeded bf16 samples of N(0, std) generated on the device (timing-only inputs), with
+    about `outlier_frac` of the entries (positions drawn with replacement) scaled x100 in
+    fp32 before the bf16 rounding, as the workloads' outliers are."""
     import torch
     g = torch.Generator(device="cuda")
     g.manual_seed(seed)
@@ -361,8 +363,18 @@ def _dev_normal(shape, std, seed):
     step = 1 << 26
     for lo in range(0, flat.numel(), step):
         hi = min(flat.numel(), lo + step)
-        flat[lo:hi] = (torch.randn(hi - lo, generator=g, device="cuda") * std).to(torch.bfloat16)
+        v = torch.randn(hi - lo, generator=g, device="cuda") * std
+        n_out = int(round(outlier_frac * (hi - lo)))
+        if n_out:
+            idx = torch.randint(0, hi - lo, (n_out,), generator=g, device="cuda")
+            v[idx] *= 100.0
+        flat[lo:hi] = v.to(torch.bfloat16)
     return out
+
+
+DEVICE_INPUTS = ("seeded device draws of the workload's shapes and distributions (N(0, std), "
+                 "0.1% x100 outliers where the workload has them); parity on the workload's own "
+                 "host-drawn inputs is covered by the GPU tests")
 
 
 def config_throughput(fq, flush_l2, reps=10):
@@ -375,8 +387,8 @@ def config_throughput(fq, flush_l2, reps=10):
     # MoE prefill: 32 experts, Zipf routing, W [4096, 7168]
     w = workloads.prefill()
     off = torch.from_numpy(w.offsets).cuda()
-    A = _dev_normal((w.M, w.K), 1.0, 3001)
-    W = _dev_normal((w.experts, w.N, w.K), 0.006, 3002)
+    A = _dev_normal((w.M, w.K), w.a_std, 3001, w.a_outliers)
+    W = _dev_normal((w.experts, w.N, w.K), w.b_std, 3002)
     qA, sA = fq.quant_act_1x128(A, False)
     qW, sW = fq.quant_weight_128x128(W, False)
     C = torch.empty((w.M, w.N), dtype=torch.bfloat16, device="cuda")
@@ -385,7 +397,7 @@ def config_throughput(fq, flush_l2, reps=10):
     t_g = _time_ms(lambda: fq.gemm_grouped(qA, sA, qW, sW, off, out=C), reps, flush_l2)
     tf = w.gemm_flops / (t_g * 1e-3) / 1e12
     out["moe_prefill"] = {
-        "workload": w.name, "sum_M": w.M, "max_M": int(w.counts.max()), "min_M": int(w.counts.min()),
+        "workload": w.name, "inputs": DEVICE_INPUTS, "sum_M": w.M, "max_M": int(w.counts.max()), "min_M": int(w.counts.min()),
         "gemm_ms": round(t_g, 4), "gemm_tflops": round(tf, 1), "gemm_frac_of_fp8_peak": round(tf / fp8_peak, 4),
         "quant_act_gbs": round(w.M * w.K * (3 + 4 / 128) / (t_a * 1e-3) / 1e9, 1),
         "quant_weight_gbs": round(W.numel() * (3 + 4 / 16384) / (t_w * 1e-3) / 1e9, 1)}
@@ -401,15 +413,15 @@ def config_throughput(fq, flush_l2, reps=10):
     # MoE decode: 64 experts, M_e ~ U{1..256}, W [7168, 2048] already FP8
     w = workloads.decode()
     off = torch.from_numpy(w.offsets).cuda()
-    A = _dev_normal((w.M, w.K), 1.0, 4001)
-    W = _dev_normal((w.experts, w.N, w.K), 0.006, 4002)
+    A = _dev_normal((w.M, w.K), w.a_std, 4001, w.a_outliers)
+    W = _dev_normal((w.experts, w.N, w.K), w.b_std, 4002)
     qA, sA = fq.quant_act_1x128(A, True)
     qW, sW = fq.quant_weight_128x128(W, False)
     C = torch.empty((w.M, w.N), dtype=torch.bfloat16, device="cuda")
     t_g = _time_ms(lambda: fq.gemm_grouped(qA, sA, qW, sW, off, out=C), reps, flush_l2)
     gemm_bytes = qW.numel() + sW.numel() * 4 + qA.numel() + sA.numel() * 4 + C.numel() * 2
     out["moe_decode"] = {
-        "workload": w.name, "sum_M": w.M, "gemm_ms": round(t_g, 4),
+        "workload": w.name, "inputs": DEVICE_INPUTS, "sum_M": w.M, "gemm_ms": round(t_g, 4),
         "gemm_tflops": round(w.gemm_flops / (t_g * 1e-3) / 1e12, 1),
         "gemm_gbs": round(gemm_bytes / (t_g * 1e-3) / 1e9, 1),
         "gemm_frac_of_hbm": round(gemm_bytes / (t_g * 1e-3) / 1e9 / hbm, 4),
@@ -424,15 +436,15 @@ def config_throughput(fq, flush_l2, reps=10):
     del A, W, qA, sA, qW, sW, C
     # wgrad: dY [7168, 16384] x X [2048, 16384], 1x128 both, fp32 out
     w = workloads.wgrad()
-    A = _dev_normal((w.M, w.K), 1e-3, 5001)
-    B = _dev_normal((w.N, w.K), 1.0, 5002)
+    A = _dev_normal((w.M, w.K), w.a_std, 5001, w.a_outliers)
+    B = _dev_normal((w.N, w.K), w.b_std, 5002)
     qA, sA = fq.quant_act_1x128(A, False)
     qB, sB = fq.quant_act_1x128(B, False)
     C = torch.empty((w.M, w.N), dtype=torch.float32, device="cuda")
     t_a = _time_ms(lambda: fq.quant_act_1x128(A, False, out=(qA, sA)), reps, flush_l2)
     t_g = _time_ms(lambda: fq.gemm_blockscaled(qA, sA, qB, sB, b_rowwise=True, out=C), reps, flush_l2)
     tf = w.gemm_flops / (t_g * 1e-3) / 1e12
-    out["wgrad"] = {"workload": w.name, "gemm_ms": round(t_g, 4), "gemm_tflops": round(tf, 1),
+    out["wgrad"] = {"workload": w.name, "inputs": DEVICE_INPUTS, "gemm_ms": round(t_g, 4), "gemm_tflops": round(tf, 1),
                     "gemm_frac_of_fp8_peak": round(tf / fp8_peak, 4),
                     "quant_act_gbs": round(w.M * w.K * (3 + 4 / 128) / (t_a * 1e-3) / 1e9, 1)}
     del A, B, qA, sA, qB, sB, C
@@ -495,17 +507,16 @@ def library_fp8_ceiling(flush_l2, n: int = 8192, reps: int = 20) -> dict:
         return {"unavailable": f"{type(e).__name__}: {str(e).splitlines()[0][:200] if str(e) else ''}"}
 
 
-def accumulation_study(fq, rows_sampled=32, w=None, ks=(4096, 8192, 16384)):
-    """Error of the promoted GEMM and of the no-promotion GEMM versus K on the wgrad
-    workload (dY [7168, K] x X [2048, K], K = 4096 / 8192 / 16384 prefixes of one draw),
-    against the float64 product of the same codes and scales on sampled rows.  Promoted:
-    1x128 codes (and, apples to apples, the 1xK codes with their row scales repeated per
-    group); no-promotion: 1xK codes, one TMEM accumulator over all of K."""
+def accumulation_study(fq, rows_sampled=128, seeds=(0, 1, 2), ks=(4096, 8192, 16384)):
+    """Error of the promoted GEMM and of the no-promotion GEMM versus K on the wgrad workload
+    (dY [7168, K] x X [2048, K], K = 4096 / 8192 / 16384 prefixes of one draw per seed),
+    against the float64 product of the same codes and scales on `rows_sampled` rows.
+    Promoted: 1x128 codes (and, apples to apples, the 1xK codes with their row scales
+    repeated per group); no-promotion: 1xK codes, one TMEM accumulator over all of K.
+    Per K: each statistic's value per seed, and its min / max over the seeds."""
     import torch
-    w = workloads.wgrad() if w is None else w
-    a_full, b_full = w.gen_a(), w.gen_b()
-    rows = np.sort(np.random.default_rng(5).choice(w.M, rows_sampled, replace=False))
-    res = []
+    w = workloads.wgrad()
+    per_seed = []
 
     def stats(Cs, C_ref, T):
         d = np.abs(Cs.astype(np.float64) - C_ref)
@@ -513,36 +524,50 @@ def accumulation_study(fq, rows_sampled=32, w=None, ks=(4096, 8192, 16384)):
         return {"max_rel_T": float(r.max()), "median_rel_T": float(np.median(r)),
                 "rel_frobenius": float(np.linalg.norm(d) / np.linalg.norm(C_ref))}
 
-    for K in ks:
-        a_bits = np.ascontiguousarray(a_full[:, :K])
-        b_bits = np.ascontiguousarray(b_full[:, :K])
-        A, B = dev_bf16(a_bits), dev_bf16(b_bits)
-        rows_t = torch.from_numpy(rows).to(A.device)
-        G = K // 128
-        qa, sa = fq.quant_act_1x128(A, False)
-        qb, sb = fq.quant_act_1x128(B, False)
-        C_p = fq.gemm_blockscaled(qa, sa, qb, sb, out_dtype=torch.float32, b_rowwise=True)
-        qa1, sa1 = fq.quant_rowwise(A)
-        qb1, sb1 = fq.quant_rowwise(B)
-        C_n = fq.gemm_nopromo(qa1, sa1, qb1, sb1)
-        C_p1 = fq.gemm_blockscaled(qa1, sa1.expand(G, -1).contiguous(), qb1,
-                                   sb1.expand(G, -1).contiguous(), out_dtype=torch.float32,
-                                   b_rowwise=True)
-        torch.cuda.synchronize()
-        # float64 products of the codes the GEMMs consumed (1xK row scales repeated per
-        # group give the 1xK codes' exact product)
-        C_ref, T = _fp64_product(qa[rows_t].cpu().numpy(), sa[:, rows_t].cpu().numpy(),
-                                 qb.cpu().numpy(), sb.cpu().numpy(), True)
-        C1_ref, T1 = _fp64_product(qa1[rows_t].cpu().numpy(),
-                                   sa1[rows_t].cpu().numpy()[None, :].repeat(G, 0),
-                                   qb1.cpu().numpy(), sb1.cpu().numpy()[None, :].repeat(G, 0), True)
-        res.append({"K": K,
-                    "promoted_1x128": stats(C_p[rows_t].cpu().numpy(), C_ref, T),
-                    "promoted_1xK_codes": stats(C_p1[rows_t].cpu().numpy(), C1_ref, T1),
-                    "no_promotion_1xK_codes": stats(C_n[rows_t].cpu().numpy(), C1_ref, T1)})
-        del A, B, qa, sa, qb, sb, C_p, qa1, sa1, qb1, sb1, C_n, C_p1
-    return {"rows_sampled": int(rows_sampled), "metric": "|C - C_ref| / sum_k|a b| (and Frobenius)",
-            "results": res}
+    for seed in seeds:
+        kmax = max(ks)
+        a_full = workloads.normal_bf16(workloads.rng_for(5, 100 + seed), (w.M, kmax), w.a_std)
+        b_full = workloads.normal_bf16(workloads.rng_for(5, 200 + seed), (w.N, kmax), w.b_std)
+        rows = np.sort(np.random.default_rng(5 + seed).choice(w.M, rows_sampled, replace=False))
+        res = []
+        for K in ks:
+            A = dev_bf16(np.ascontiguousarray(a_full[:, :K]))
+            B = dev_bf16(np.ascontiguousarray(b_full[:, :K]))
+            rows_t = torch.from_numpy(rows).to(A.device)
+            G = K // 128
+            qa, sa = fq.quant_act_1x128(A, False)
+            qb, sb = fq.quant_act_1x128(B, False)
+            C_p = fq.gemm_blockscaled(qa, sa, qb, sb, out_dtype=torch.float32, b_rowwise=True)
+            qa1, sa1 = fq.quant_rowwise(A)
+            qb1, sb1 = fq.quant_rowwise(B)
+            C_n = fq.gemm_nopromo(qa1, sa1, qb1, sb1)
+            C_p1 = fq.gemm_blockscaled(qa1, sa1.expand(G, -1).contiguous(), qb1,
+                                       sb1.expand(G, -1).contiguous(), out_dtype=torch.float32,
+                                       b_rowwise=True)
+            torch.cuda.synchronize()
+            C_ref, T = _fp64_product(qa[rows_t].cpu().numpy(), sa[:, rows_t].cpu().numpy(),
+                                     qb.cpu().numpy(), sb.cpu().numpy(), True)
+            C1_ref, T1 = _fp64_product(qa1[rows_t].cpu().numpy(),
+                                       sa1[rows_t].cpu().numpy()[None, :].repeat(G, 0),
+                                       qb1.cpu().numpy(), sb1.cpu().numpy()[None, :].repeat(G, 0), True)
+            res.append({"K": K,
+                        "promoted_1x128": stats(C_p[rows_t].cpu().numpy(), C_ref, T),
+                        "promoted_1xK_codes": stats(C_p1[rows_t].cpu().numpy(), C1_ref, T1),
+                        "no_promotion_1xK_codes": stats(C_n[rows_t].cpu().numpy(), C1_ref, T1)})
+            del A, B, qa, sa, qb, sb, C_p, qa1, sa1, qb1, sb1, C_n, C_p1
+        per_seed.append(res)
+    summary = []
+    for i, K in enumerate(ks):
+        entry = {"K": K}
+        for path in ("promoted_1x128", "promoted_1xK_codes", "no_promotion_1xK_codes"):
+            entry[path] = {}
+            for stat in ("max_rel_T", "median_rel_T", "rel_frobenius"):
+                vals = [per_seed[j][i][path][stat] for j in range(len(seeds))]
+                entry[path][stat] = {"per_seed": vals, "min": min(vals), "max": max(vals)}
+        summary.append(entry)
+    return {"rows_sampled": int(rows_sampled), "seeds": list(seeds),
+            "metric": "|C - C_ref| / sum_k|a b| (max, median) and relative Frobenius error",
+            "results": summary}
 
 
 def profile_case(args, name: str, launches: int = 3):

@@ -145,10 +145,14 @@ struct GemmCfg {
   static constexpr uint32_t a = 0;
   static constexpr uint32_t b = a + kStages * kABytes;
   static constexpr uint32_t bars = b + kStages * kBBytes;
-  // Scale ring: a slot holds one group's 128 A row scales and its B scales (the tile's
-  // kN column scales in ROW mode; its kN / 128 block scales, padded to 4, otherwise).
-  static constexpr int kScaleSlots = ROW_B ? 16 : 24;
-  static constexpr uint32_t kSlotFloats = 128 + (ROW_B ? kN : 4);
+  // Scale ring: a slot holds the scales of kSlotGroups consecutive groups of the CTA's
+  // stream; per group its 128 A row scales and its B scales (the tile's kN column scales
+  // in ROW mode; its kN / 128 block scales, padded to 4, otherwise).  One barrier wait
+  // and one release per slot, not per group.
+  static constexpr int kSlotGroups = 4;
+  static constexpr int kScaleSlots = ROW_B ? 4 : 6;
+  static constexpr uint32_t kGroupFloats = 128 + (ROW_B ? kN : 4);
+  static constexpr uint32_t kSlotFloats = kSlotGroups * kGroupFloats;
   // full[S], empty[S], tfull[NB], tempty[NB], drain, sfull[R], sempty[R]
   static constexpr uint32_t n_bars = 2 * kStages + 2 * kAccBufs + 1 + 2 * kScaleSlots;
   static constexpr uint32_t misc = align_up(bars + 8 * n_bars, 16);   // tmem slot, abort flag
@@ -159,7 +163,7 @@ struct GemmCfg {
   static constexpr uint32_t smem_bytes = end + 1024;                  // + base alignment slack
   static_assert(a % 1024 == 0 && b % 1024 == 0 && kABytes % 1024 == 0 && kBBytes % 1024 == 0,
                 "swizzle atoms");
-  static_assert(sbrow % 16 == 0 && sring % 16 == 0 && kSlotFloats % 4 == 0 && kN / 128 <= 4,
+  static_assert(sbrow % 16 == 0 && sring % 16 == 0 && kGroupFloats % 4 == 0 && kN / 128 <= 4,
                 "float4 reads of the scale slots");
   static_assert(kSetCols % 64 == 0 && kAccBufs >= 2, "64-column loads; two accumulators");
   static_assert(kN % 16 == 0 && kN <= 256 && kBBox <= 256, "MMA N and TMA box");
@@ -408,6 +412,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // Slot layout: [0, 128) A scales of the tile's 128 rows; then the B scales: the
       // tile's kN column scales (ROW mode) or, for 128x128 weight blocks, the kN / 128
       // blocks' scales.
+      // `it` counts the CTA's groups; group it goes to slot (it / kSlotGroups) % R, part
+      // it % kSlotGroups.  A slot is published after its last group, or after the CTA's
+      // last group when that slot is only partly filled.
+      constexpr uint32_t SG = Cfg::kSlotGroups;
       uint32_t it = 0;
       bool ok = true;
       for (int ui = 0; ok && ui < n_units; ++ui) {
@@ -416,12 +424,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const float* sB_tile =
             ROW_B ? nullptr : p.sB + (static_cast<int64_t>(tl.expert) * (p.N / 128) + tl.col0 / 128) * G;
         for (int g = u.g0; g < u.g1; ++g, ++it) {
-          const int r = it % R;
-          if (!mbar_wait(sempty_bar(r), ((it / R) & 1u) ^ 1u, kSiteScales, abort_flag)) {
+          const uint32_t sl = it / SG;
+          const int r = sl % R;
+          if (it % SG == 0 &&
+              !mbar_wait(sempty_bar(r), ((sl / R) & 1u) ^ 1u, kSiteScales, abort_flag)) {
             ok = false;
             break;
           }
-          const uint32_t slot = sbase + Cfg::sring + 4u * Cfg::kSlotFloats * r;
+          const uint32_t slot = sbase + Cfg::sring + 4u * (Cfg::kSlotFloats * r + Cfg::kGroupFloats * (it % SG));
           const float* sa_g = p.sA + static_cast<int64_t>(g) * p.ld_sa;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -439,9 +449,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const bool v = tl.col0 + 128 * lane < p.N;
             cp_async_4(slot + 4u * (128 + lane), sB_tile + (v ? lane * G + g : 0), v);
           }
-          cp_async_arrive(sfull_bar(r));
+          if (it % SG == SG - 1) cp_async_arrive(sfull_bar(r));
         }
       }
+      if (ok && it % SG != 0) cp_async_arrive(sfull_bar((it / SG) % R));   // the last, partial slot
       cp_async_wait_all();     // no copy into shared memory outlives the CTA
     }
   } else {
@@ -483,9 +494,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int g = u.g0; g < u.g1; ++g) {
           // This group's scales, staged by the scale producer (the ring advances with
           // every group of every tile, in the same order as acc_it).
-          const int r = acc_it % R;
-          const int slot = Cfg::kSlotFloats * r;
-          if (ok) ok = mbar_wait(sfull_bar(r), (acc_it / R) & 1u, kSiteScales, abort_flag);
+          constexpr uint32_t SG = Cfg::kSlotGroups;
+          const uint32_t sl = acc_it / SG;
+          const int r = sl % R;
+          const int slot = Cfg::kSlotFloats * r + Cfg::kGroupFloats * (acc_it % SG);
+          if (ok && acc_it % SG == 0) ok = mbar_wait(sfull_bar(r), (sl / R) & 1u, kSiteScales, abort_flag);
           const float sa_cur = sring[slot + quad * 32 + lane];
           const float sb_cur = ROW_B ? 0.0f : sring[slot + 128 + set * kSetCols / 128];
           const int sb = slot + 128 + set * kSetCols;        // ROW mode column scales
@@ -509,7 +522,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           } else if (ok) {
             release(buf);
           }
-          mbar_arrive(sempty_bar(r));   // scales of this group consumed
+          if (acc_it % SG == SG - 1) mbar_arrive(sempty_bar(r));   // the slot's groups consumed
           ++acc_it;
         }
       } else {
