@@ -361,16 +361,29 @@ int fp8q_quant_act_dual(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
       return FP8Q_ERR_CUDA;
     ready.fetch_or(1ull << dev, std::memory_order_acq_rel);
   }
+  // the bf16 tile arrives by TMA: boxes of 128 rows x 64 columns, 128-byte swizzle
+  CUtensorMap tmx;
+  {
+    auto enc = tensor_map_encoder();
+    if (!enc || !bind_current_context()) return FP8Q_ERR_CUDA;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldx) * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estr[2] = {1, 1};
+    if (enc(&tmx, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return FP8Q_ERR_CUDA;
+  }
   const unsigned grid = static_cast<unsigned>((M / 128) * (K / 128));
   const auto g32 = static_cast<uint32_t>(K / 128);
   auto stm = static_cast<cudaStream_t>(stream);
-  const auto* xs = static_cast<const uint16_t*>(x);
   if (pow2_scale)
-    fp8q::quant_act_dual_kernel<true><<<grid, 256, fp8q::kDualSmem, stm>>>(xs, ldx, q, ldq, s, ld_s, qt,
-                                                                           ldqt, st, ld_st, g32);
+    fp8q::quant_act_dual_kernel<true><<<grid, 256, fp8q::kDualSmem, stm>>>(tmx, q, ldq, s, ld_s, qt, ldqt,
+                                                                           st, ld_st, g32);
   else
-    fp8q::quant_act_dual_kernel<false><<<grid, 256, fp8q::kDualSmem, stm>>>(xs, ldx, q, ldq, s, ld_s, qt,
-                                                                            ldqt, st, ld_st, g32);
+    fp8q::quant_act_dual_kernel<false><<<grid, 256, fp8q::kDualSmem, stm>>>(tmx, q, ldq, s, ld_s, qt, ldqt,
+                                                                            st, ld_st, g32);
   return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 

@@ -230,146 +230,199 @@ __global__ void __launch_bounds__(256) quant_act_1x128_kernel(const uint16_t* __
 //
 // Grid (M/128 * K/128), 256 threads, one 128x128 tile of X per block, the column group
 // running fastest (block b: group b % (K/128) of row tile b / (K/128), as for the 1x128
-// kernel):
-//  rows:    as quant_act_1x128_kernel (teams of 4 lanes per row, 16 rows per warp), all
-//           eight 16-byte loads of a thread in flight before any arithmetic; the tile is
-//           kept in shared memory with a 320-byte row pitch (the two rows a quarter-warp
-//           stores land 16 banks apart);
-//  columns: thread t owns the column pair 2 (t % 64), +1 and rows 32 (t / 64) .. + 31,
-//           read once into registers (32-bit shared loads); the four quarters' amax meet
-//           in shared memory; the codes are staged transposed in the tile's space once
-//           every thread has read it (row pitch kDualPitch bytes) and written as 128-byte
-//           column segments.  4 CTAs per SM (the 32 column words live in registers).
-constexpr int kDualPitch = 144;                     // 128 codes + 16
-constexpr int kDualRowPitch = 320;                 // bf16 tile rows: alternate rows 16 banks apart
-constexpr int kDualSmem = 128 * kDualRowPitch + 4 * 64 * 4;   // tile (reused for the codes) + amax parts
-static_assert(128 * kDualPitch <= 128 * kDualRowPitch, "codes fit in the tile's space");
+// kernel).  The tile comes into shared memory by TMA (two boxes of 128 rows x 64 columns,
+// 128-byte swizzle: 16-byte chunk c of row r of a box at chunk c ^ (r % 8)), so no
+// registers hold it in flight and 6 CTAs fit on an SM: while some quantize, others load.
+//  rows:    teams of 4 lanes per row (16 rows per warp), each lane 4 of the row's 16
+//           chunks; odd rows take their chunks rotated by 4, so the 8 chunks one phase of a
+//           16-byte shared load reads fall in 8 different bank groups under the swizzle.
+//  columns: warp w owns columns 16 w .. 16 w + 15.  ldmatrix.x4.trans hands lane i, for
+//           each of its two column blocks of 8, column i / 4 of the block in rows
+//           8 b + 2 (i % 4), +1 of every 8-row block b: 32 rows per lane, the four lanes
+//           of a quad cover the 128 (8 rows with one logical chunk are 8 swizzled chunks:
+//           no bank conflicts).  The column amax is two shuffles inside the quad; the
+//           codes are made two rows at a time (f32x2 quotients, one cvt per pair) and a
+//           4x4 transpose of 32-bit words inside the quad gives each lane whole 16-row
+//           segments of a column, written as 16-byte stores.
+constexpr int kDualTileBytes = 128 * 128 * 2;      // bf16 tile: two 16 KB boxes
+constexpr int kDualSmem = kDualTileBytes + 16 + 1024;   // + mbarrier + 1024-byte alignment
+constexpr unsigned int kSiteDual = 9;               // error site of the tile wait
 
-template <bool POW2>
-__device__ __forceinline__ void quant_act_dual_tile(const uint16_t* __restrict__ x, int64_t ldx,
-                                                    uint8_t* __restrict__ q, int64_t ldq,
-                                                    float* __restrict__ s, int64_t lds,
-                                                    uint8_t* __restrict__ qt, int64_t ldqt,
-                                                    float* __restrict__ st, int64_t ldst,
-                                                    int64_t rb, int64_t g) {
-  extern __shared__ __align__(16) uint8_t dual_smem[];
-  uint8_t* tile = dual_smem;                               // bf16 [128][128], then E4M3 codes
-  uint32_t* part = reinterpret_cast<uint32_t*>(dual_smem + 128 * kDualRowPitch);   // [4][64] amax pairs
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int l4 = lane & 3;
-  const int64_t m0 = rb * 128;
-  const int64_t k0 = g * 128;
+// Shared address of 16-byte chunk c (0..15) of tile row r (the TMA box layout).
+__device__ __forceinline__ uint32_t dual_chunk(uint32_t tile, uint32_t r, uint32_t c) {
+  return tile + (c >> 3) * (128u * 128u) + r * 128u + (((c & 7u) ^ (r & 7u)) << 4);
+}
 
-  // ---- rows: both passes' loads first
-  uint4 v[2][4];
-#pragma unroll
-  for (int pass = 0; pass < 2; ++pass) {
-    const int64_t m = m0 + warp * 16 + pass * 8 + (lane >> 2);
-    const uint16_t* src = x + m * ldx + k0 + l4 * 8;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) v[pass][j] = ldg_stream(src + 32 * j);
+// x / s for two values, one rule of Quotient each, f32x2 where the rule allows.  A pass
+// picks the rule once per warp (every lane's tile agrees on it: a vote), so the loops
+// carry no per-element branches; the general form remains for warps whose tiles differ.
+struct PairExact {              // s a power of two: x * (1/s) exactly
+  float2 r2;
+  __device__ __forceinline__ explicit PairExact(const Quotient& q) : r2(make_float2(q.r, q.r)) {}
+  __device__ __forceinline__ float2 operator()(float2 x) const { return __fmul2_rn(x, r2); }
+};
+struct PairCorrected {          // Markstein's correction with the rounded reciprocal
+  float2 r2, ns2;
+  __device__ __forceinline__ explicit PairCorrected(const Quotient& q)
+      : r2(make_float2(q.r, q.r)), ns2(make_float2(-q.s, -q.s)) {}
+  __device__ __forceinline__ float2 operator()(float2 x) const {
+    const float2 q0 = __fmul2_rn(x, r2);
+    const float2 e = __ffma2_rn(q0, ns2, x);    // x - q0 s, exact
+    const float2 y = __ffma2_rn(e, r2, q0);
+    return make_float2(copysignf(y.x, x.x), copysignf(y.y, x.y));
   }
-#pragma unroll
-  for (int pass = 0; pass < 2; ++pass) {
-    const int r = warp * 16 + pass * 8 + (lane >> 2);      // row inside the tile
-    const int64_t m = m0 + r;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(tile + r * kDualRowPitch + (l4 + 4 * j) * 16) = v[pass][j];
-    float a = amax_vectors(v[pass]);
-    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
-    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
-    const float sc = tile_scale(a, POW2);
-    const Quotient qd(sc);
-    uint2 o[4];
-    quant_vectors(v[pass], qd, o);
-    uint8_t* dst = q + m * ldq + k0 + l4 * 8;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) stg_u2(dst + 32 * j, o[j]);
-    if (l4 == 0) s[g * lds + m] = sc;
-  }
-  __syncthreads();
+};
+struct PairGeneral {            // any rule, decided per call
+  Quotient q;
+  __device__ __forceinline__ explicit PairGeneral(const Quotient& q_) : q(q_) {}
+  __device__ __forceinline__ float2 operator()(float2 x) const { return make_float2(q(x.x), q(x.y)); }
+};
 
-  // ---- columns 2p, 2p+1 over rows 32h .. 32h + 31
-  const int p = threadIdx.x & 63, h = threadIdx.x >> 6;
-  const uint32_t* words = reinterpret_cast<const uint32_t*>(tile) + p;   // row r: words[80 r]
-  uint32_t wv[32];
-  uint32_t mx = 0;
+// Runs body(pair quotient of the calling lane's tile) with the rule picked once per warp.
+template <typename Body>
+__device__ __forceinline__ void with_pair_quotient(const Quotient& q, Body body) {
+  if (__all_sync(0xffffffffu, q.mode == kCorrected)) body(PairCorrected(q));
+  else if (__all_sync(0xffffffffu, q.mode == kExactRcp)) body(PairExact(q));
+  else body(PairGeneral(q));
+}
+
+// In-quad 4x4 transpose of 32-bit words: lane q of a group of 4 lanes holds row q of a
+// 4x4 matrix in v[0..3]; afterwards it holds column q.  Two exchange stages (partners
+// q ^ 1, then q ^ 2), two shuffles each.
+__device__ __forceinline__ void quad_transpose4(uint32_t (&v)[4], int q) {
 #pragma unroll
-  for (int r = 0; r < 32; ++r) {
-    wv[r] = words[(32 * h + r) * (kDualRowPitch / 4)];
-    mx = __vmaxu2(mx, wv[r] & 0x7FFF7FFFu);
+  for (int t = 0; t < 2; ++t) {            // 2x2 blocks: swap the off-diagonal elements
+    const bool odd = q & 1;
+    const uint32_t send = odd ? v[2 * t] : v[2 * t + 1];
+    const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, 1);
+    if (odd) v[2 * t] = recv; else v[2 * t + 1] = recv;
   }
-  part[h * 64 + p] = mx;
-  __syncthreads();
-  const uint32_t mall = __vmaxu2(__vmaxu2(part[p], part[64 + p]), __vmaxu2(part[128 + p], part[192 + p]));
-  const float sc_lo = tile_scale(__uint_as_float((mall & 0xFFFFu) << 16), POW2);
-  const float sc_hi = tile_scale(__uint_as_float(mall & 0xFFFF0000u), POW2);
-  const Quotient q_lo(sc_lo), q_hi(sc_hi);
-  uint32_t c_lo[8], c_hi[8];                               // 32 codes of each column
-  // the quotient rule is picked once for the pair (both columns share it but for rare
-  // scales that happen to be powers of two, or tiny ones)
-  auto codes_with = [&](auto f_lo, auto f_hi) {
 #pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      const uint32_t w0 = wv[4 * w], w1 = wv[4 * w + 1];
-      const uint32_t w2 = wv[4 * w + 2], w3 = wv[4 * w + 3];
-      c_lo[w] = cvt_e4m3x2(f_lo(bf16lo(w0)), f_lo(bf16lo(w1))) |
-                (cvt_e4m3x2(f_lo(bf16lo(w2)), f_lo(bf16lo(w3))) << 16);
-      c_hi[w] = cvt_e4m3x2(f_hi(bf16hi(w0)), f_hi(bf16hi(w1))) |
-                (cvt_e4m3x2(f_hi(bf16hi(w2)), f_hi(bf16hi(w3))) << 16);
-    }
-  };
-  if (q_lo.mode == kCorrected && q_hi.mode == kCorrected) {
-    const float r_lo = q_lo.r, s_lo = q_lo.s, r_hi = q_hi.r, s_hi = q_hi.s;
-    codes_with(
-        [r_lo, s_lo](float xv) {
-          const float q0 = __fmul_rn(xv, r_lo);
-          return copysignf(__fmaf_rn(__fmaf_rn(-q0, s_lo, xv), r_lo, q0), xv);
-        },
-        [r_hi, s_hi](float xv) {
-          const float q0 = __fmul_rn(xv, r_hi);
-          return copysignf(__fmaf_rn(__fmaf_rn(-q0, s_hi, xv), r_hi, q0), xv);
-        });
-  } else if (q_lo.mode == kExactRcp && q_hi.mode == kExactRcp) {
-    const float r_lo = q_lo.r, r_hi = q_hi.r;
-    codes_with([r_lo](float xv) { return __fmul_rn(xv, r_lo); },
-               [r_hi](float xv) { return __fmul_rn(xv, r_hi); });
-  } else {
-    codes_with([&q_lo](float xv) { return q_lo(xv); }, [&q_hi](float xv) { return q_hi(xv); });
-  }
-  if (h == 0) {
-    float* sdst = st + (m0 / 128) * ldst + k0 + 2 * p;
-    sdst[0] = sc_lo;
-    sdst[1] = sc_hi;
-  }
-  __syncthreads();                                         // every thread is done reading the tile
-  uint8_t* codes = tile;                                   // [128 columns][kDualPitch]
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    *reinterpret_cast<uint4*>(codes + (2 * p) * kDualPitch + 32 * h + 16 * j) =
-        make_uint4(c_lo[4 * j], c_lo[4 * j + 1], c_lo[4 * j + 2], c_lo[4 * j + 3]);
-    *reinterpret_cast<uint4*>(codes + (2 * p + 1) * kDualPitch + 32 * h + 16 * j) =
-        make_uint4(c_hi[4 * j], c_hi[4 * j + 1], c_hi[4 * j + 2], c_hi[4 * j + 3]);
-  }
-  __syncthreads();
-  // 128 columns x 128 codes: each group of 8 threads writes one 128-byte column segment
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int idx = j * 256 + threadIdx.x;
-    const int cc = idx >> 3, chunk = idx & 7;
-    const uint4 val = *reinterpret_cast<const uint4*>(codes + cc * kDualPitch + chunk * 16);
-    *reinterpret_cast<uint4*>(qt + (k0 + cc) * ldqt + m0 + chunk * 16) = val;
+  for (int t = 0; t < 2; ++t) {            // swap the off-diagonal 2x2 blocks
+    const bool hi = q & 2;
+    const uint32_t send = hi ? v[t] : v[2 + t];
+    const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, 2);
+    if (hi) v[t] = recv; else v[2 + t] = recv;
   }
 }
 
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                                  uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr)
+               : "memory");
+}
+
 template <bool POW2>
-__global__ void __launch_bounds__(256, 4) quant_act_dual_kernel(const uint16_t* __restrict__ x,
-                                                             int64_t ldx, uint8_t* __restrict__ q,
-                                                             int64_t ldq, float* __restrict__ s,
-                                                             int64_t lds, uint8_t* __restrict__ qt,
-                                                             int64_t ldqt, float* __restrict__ st,
-                                                             int64_t ldst, uint32_t G) {
-  quant_act_dual_tile<POW2>(x, ldx, q, ldq, s, lds, qt, ldqt, st, ldst, blockIdx.x / G, blockIdx.x % G);
+__global__ void __launch_bounds__(256, 6) quant_act_dual_kernel(const __grid_constant__ CUtensorMap tmx,
+                                                             uint8_t* __restrict__ q, int64_t ldq,
+                                                             float* __restrict__ s, int64_t lds,
+                                                             uint8_t* __restrict__ qt, int64_t ldqt,
+                                                             float* __restrict__ st, int64_t ldst,
+                                                             uint32_t G) {
+  extern __shared__ uint8_t dual_raw[];
+  const uint32_t tile = (smem_u32(dual_raw) + 1023u) & ~1023u;   // swizzle atoms need 1 KB
+  const uint32_t bar = tile + kDualTileBytes;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int l4 = lane & 3;
+  const int64_t g = blockIdx.x % G, m0 = static_cast<int64_t>(blockIdx.x / G) * 128;
+  const int64_t k0 = g * 128;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(bar, kDualTileBytes);
+    tma_load_2d(tile, &tmx, bar, static_cast<int32_t>(k0), static_cast<int32_t>(m0));
+    tma_load_2d(tile + kDualTileBytes / 2, &tmx, bar, static_cast<int32_t>(k0 + 64), static_cast<int32_t>(m0));
+  }
+  // bounded (the loads end on their own); a timeout is recorded and the tile skipped
+  if (!__syncthreads_and(mbar_wait(bar, 0, kSiteDual, nullptr))) return;
+
+  // ---- rows: lane l4 of the team of row r holds chunks (l4 + 4 j + 4 (r & 1)) % 16
+#pragma unroll
+  for (int pass = 0; pass < 2; ++pass) {
+    const uint32_t r = warp * 16 + pass * 8 + (lane >> 2);  // row inside the tile
+    const int64_t m = m0 + r;
+    uint4 v[4];
+    uint32_t cj[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      cj[j] = (l4 + 4 * j + 4 * (r & 1)) & 15u;
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(v[j].x), "=r"(v[j].y), "=r"(v[j].z), "=r"(v[j].w)
+                   : "r"(dual_chunk(tile, r, cj[j])));
+    }
+    float a = amax_vectors(v);
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+    const float sc = tile_scale(a, POW2);
+    uint8_t* dst = q + m * ldq + k0;
+    with_pair_quotient(Quotient(sc), [&](const auto& qd) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 w = v[j];
+        const float2 p0 = qd(make_float2(bf16lo(w.x), bf16hi(w.x)));
+        const float2 p1 = qd(make_float2(bf16lo(w.y), bf16hi(w.y)));
+        const float2 p2 = qd(make_float2(bf16lo(w.z), bf16hi(w.z)));
+        const float2 p3 = qd(make_float2(bf16lo(w.w), bf16hi(w.w)));
+        uint2 o;
+        o.x = __byte_perm(cvt_e4m3x2(p0.x, p0.y), cvt_e4m3x2(p1.x, p1.y), 0x5410);
+        o.y = __byte_perm(cvt_e4m3x2(p2.x, p2.y), cvt_e4m3x2(p3.x, p3.y), 0x5410);
+        stg_u2(dst + 8 * cj[j], o);
+      }
+    });
+    if (l4 == 0) s[g * lds + m] = sc;
+  }
+
+  // ---- columns 16 warp + 8 h + lane / 4 (h = 0, 1), all 128 rows
+  const int quad = lane >> 2;                  // column inside the 8-column block
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t chunk = static_cast<uint32_t>(2 * warp + h);    // 16-byte chunk of the rows
+    // lane l addresses row 8 (rb4 + l / 8) + l % 8 of 4 consecutive 8-row blocks
+    uint32_t w2[16];                           // w2[b]: rows 8b + 2 l4, +1 of the column
+#pragma unroll
+    for (int rb4 = 0; rb4 < 16; rb4 += 4) {
+      const uint32_t r = static_cast<uint32_t>(8 * (rb4 + (lane >> 3)) + (lane & 7));
+      ldmatrix_x4_trans(dual_chunk(tile, r, chunk), w2[rb4], w2[rb4 + 1], w2[rb4 + 2], w2[rb4 + 3]);
+    }
+    uint32_t mx = 0;
+#pragma unroll
+    for (int b = 0; b < 16; ++b) mx = __vmaxu2(mx, w2[b] & 0x7FFF7FFFu);
+    float a = __uint_as_float(((mx >> 16) > (mx & 0xFFFFu) ? (mx >> 16) : (mx & 0xFFFFu)) << 16);
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+    const float sc = tile_scale(a, POW2);
+    // pairs of codes: rows 8b + 2 l4 (low byte) and 8b + 2 l4 + 1
+    uint32_t vv[8];                            // vv[c]: rows 16c + 2 l4, +1 | 16c + 8 + 2 l4, +1
+    with_pair_quotient(Quotient(sc), [&](const auto& qd) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float2 e0 = qd(make_float2(bf16lo(w2[2 * c]), bf16hi(w2[2 * c])));
+        const float2 e1 = qd(make_float2(bf16lo(w2[2 * c + 1]), bf16hi(w2[2 * c + 1])));
+        vv[c] = __byte_perm(cvt_e4m3x2(e0.x, e0.y), cvt_e4m3x2(e1.x, e1.y), 0x5410);
+      }
+    });
+    // lane l4 of the quad gathers 16-row segments l4 and l4 + 4 of the column
+    uint32_t lo[4] = {vv[0], vv[1], vv[2], vv[3]};
+    uint32_t hi4[4] = {vv[4], vv[5], vv[6], vv[7]};
+    quad_transpose4(lo, l4);
+    quad_transpose4(hi4, l4);
+    const int64_t col = k0 + 16 * warp + 8 * h + quad;
+    uint8_t* row = qt + col * ldqt + m0;
+    // from lane j of the quad: rows 2j, 2j+1 (low half) and 8 + 2j, 9 + 2j (high half)
+    *reinterpret_cast<uint4*>(row + 16 * l4) =
+        make_uint4(__byte_perm(lo[0], lo[1], 0x5410), __byte_perm(lo[2], lo[3], 0x5410),
+                   __byte_perm(lo[0], lo[1], 0x7632), __byte_perm(lo[2], lo[3], 0x7632));
+    *reinterpret_cast<uint4*>(row + 16 * (l4 + 4)) =
+        make_uint4(__byte_perm(hi4[0], hi4[1], 0x5410), __byte_perm(hi4[2], hi4[3], 0x5410),
+                   __byte_perm(hi4[0], hi4[1], 0x7632), __byte_perm(hi4[2], hi4[3], 0x7632));
+    if (l4 == 0) st[(m0 / 128) * ldst + col] = sc;
+  }
 }
 
 // ---------------------------------------------------------------- transposed weight blocks

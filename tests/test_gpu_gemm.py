@@ -227,6 +227,13 @@ def test_grouped_ragged_with_slack_rows(fq, out_fp32):
                   alloc_rows=4096)
 
 
+@pytest.mark.parametrize("out_fp32", [True, False])
+def test_grouped_decode_expert_sizes(fq, out_fp32):
+    """Experts of 1, 16, 128, 129 and 256 tokens: one and two row tiles, nearly empty and
+    full ones."""
+    _grouped_case(fq, [1, 16, 128, 129, 256], 384, 512, True, out_fp32, seed=41, name="expert sizes")
+
+
 def test_grouped_unwritten_rows_untouched(fq):
     """Rows past the last offset (allocation slack) are not written."""
     import torch
