@@ -507,15 +507,16 @@ def library_fp8_ceiling(flush_l2, n: int = 8192, reps: int = 20) -> dict:
         return {"unavailable": f"{type(e).__name__}: {str(e).splitlines()[0][:200] if str(e) else ''}"}
 
 
-def accumulation_study(fq, rows_sampled=128, seeds=(0, 1, 2), ks=(4096, 8192, 16384)):
+def accumulation_study(fq, rows_sampled=128, seeds=(0, 1, 2), ks=(4096, 8192, 16384), w=None):
     """Error of the promoted GEMM and of the no-promotion GEMM versus K on the wgrad workload
     (dY [7168, K] x X [2048, K], K = 4096 / 8192 / 16384 prefixes of one draw per seed),
     against the float64 product of the same codes and scales on `rows_sampled` rows.
     Promoted: 1x128 codes (and, apples to apples, the 1xK codes with their row scales
     repeated per group); no-promotion: 1xK codes, one TMEM accumulator over all of K.
-    Per K: each statistic's value per seed, and its min / max over the seeds."""
+    Per K: each statistic's value per seed, and its min / max over the seeds.  `w`: the
+    shapes and spreads to draw (default: the wgrad workload)."""
     import torch
-    w = workloads.wgrad()
+    w = workloads.wgrad() if w is None else w
     per_seed = []
 
     def stats(Cs, C_ref, T):

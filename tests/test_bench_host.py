@@ -136,15 +136,15 @@ def test_accumulation_study_runs_on_host_stand_ins(monkeypatch):
     monkeypatch.setattr(bench, "dev_bf16",
                         lambda b: t(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16))
     monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
-    rng = np.random.default_rng(14)
-    a = workloads.normal_bf16(rng, (96, 512), 1e-3)
-    b = workloads.normal_bf16(rng, (256, 512), 1.0)
-    w = SimpleNamespace(M=96, gen_a=lambda: a, gen_b=lambda: b)
-    res = bench.accumulation_study(fake, rows_sampled=8, w=w, ks=(256, 512))
-    assert res["rows_sampled"] == 8 and [r["K"] for r in res["results"]] == [256, 512]
+    w = SimpleNamespace(M=96, N=256, a_std=1e-3, b_std=1.0)
+    res = bench.accumulation_study(fake, rows_sampled=8, seeds=(0, 1), ks=(256, 512), w=w)
+    assert res["rows_sampled"] == 8 and res["seeds"] == [0, 1]
+    assert [r["K"] for r in res["results"]] == [256, 512]
     for r in res["results"]:
         for key in ("promoted_1x128", "promoted_1xK_codes", "no_promotion_1xK_codes"):
-            assert 0 <= r[key]["max_rel_T"] < 1e-7 and r[key]["rel_frobenius"] < 1e-6
+            mx, fro = r[key]["max_rel_T"], r[key]["rel_frobenius"]
+            assert len(mx["per_seed"]) == 2 and mx["min"] <= mx["max"]
+            assert 0 <= mx["max"] < 1e-7 and fro["max"] < 1e-6
     json.dumps(res)
 
 
