@@ -65,11 +65,13 @@ __device__ __forceinline__ float tile_scale(float amax, bool pow2) {
 // Three ways, chosen once per tile (uniform across the threads of the tile):
 //  kExactRcp: s is a power of two >= 2^-126, so 1/s is exact and x * (1/s) is x / s.
 //  kCorrected: s >= 2^-92.  r = RN(1/s); q0 = RN(x r) is within one ulp of x/s; the
-//    residual x - q0 s is exact under one FMA; RN(q0 + residual r) is RN(x / s)
-//    (Markstein's correction with a correctly rounded reciprocal).  For quotients
-//    below 2^-11 the residual may lose bits, but such quotients round to a signed
-//    zero in E4M3 either way; copysign keeps the sign of x for x = -0.  An
-//    exhaustive host check over every bf16 pair (amax, x) backs this.
+//    residual is exact under one FMA; RN(q0 + residual r) is RN(x / s) (Markstein's
+//    correction with a correctly rounded reciprocal).  The residual is taken with the
+//    opposite sign, d = q0 s - x, and the quotient as RN(q0 - d r): the same values,
+//    but for x = -0 (q0 = -0, d = +0) the last step adds -0 to -0 and keeps the sign, so
+//    no sign restore is needed.  For quotients below 2^-11 the residual may lose bits,
+//    but such quotients round to a signed zero in E4M3 either way.  An exhaustive host
+//    check over every bf16 pair (amax, x) backs this.
 //  kDivide: IEEE division (tiny scales).
 enum QuotMode { kExactRcp = 0, kCorrected = 1, kDivide = 2 };
 
@@ -93,8 +95,8 @@ struct Quotient {
     if (mode == kExactRcp) return __fmul_rn(x, r);
     if (mode == kCorrected) {
       const float q0 = __fmul_rn(x, r);
-      const float e = __fmaf_rn(-q0, s, x);
-      return copysignf(__fmaf_rn(e, r, q0), x);
+      const float d = __fmaf_rn(q0, s, -x);
+      return __fmaf_rn(d, -r, q0);
     }
     return __fdiv_rn(x, s);
   }
@@ -102,6 +104,12 @@ struct Quotient {
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+// The negated values (-x) of the low / high bf16 of a word: one integer op each, with the
+// sign flip folded in (adding 2^31 flips bit 31).
+__device__ __forceinline__ float bf16lo_neg(uint32_t w) { return __uint_as_float(w * 65536u + 0x80000000u); }
+__device__ __forceinline__ float bf16hi_neg(uint32_t w) {
+  return __uint_as_float((w & 0xFFFF0000u) ^ 0x80000000u);
+}
 
 // 8 bf16 -> 8 E4M3 bytes (uint2), each divided by the tile scale with quotient rule Q.
 template <typename Q>
@@ -124,8 +132,8 @@ __device__ __forceinline__ void quant_vectors(const uint4 (&v)[NV], const Quotie
     const float r = qd.r, sc = qd.s;
     auto f = [r, sc](float x) {
       const float q0 = __fmul_rn(x, r);
-      const float e = __fmaf_rn(-q0, sc, x);
-      return copysignf(__fmaf_rn(e, r, q0), x);
+      const float d = __fmaf_rn(q0, sc, -x);
+      return __fmaf_rn(d, -r, q0);
     };
 #pragma unroll
     for (int j = 0; j < NV; ++j) o[j] = quant8_with(v[j], f);
@@ -256,26 +264,28 @@ __device__ __forceinline__ uint32_t dual_chunk(uint32_t tile, uint32_t r, uint32
 // x / s for two values, one rule of Quotient each, f32x2 where the rule allows.  A pass
 // picks the rule once per warp (every lane's tile agrees on it: a vote), so the loops
 // carry no per-element branches; the general form remains for warps whose tiles differ.
+// Pair quotients take the NEGATED pair nx = (-x0, -x1) (bf16lo_neg / bf16hi_neg) and
+// return (x0 / s, x1 / s) rounded as Quotient does; the f32x2 instructions then need no
+// operand negation.
 struct PairExact {              // s a power of two: x * (1/s) exactly
-  float2 r2;
-  __device__ __forceinline__ explicit PairExact(const Quotient& q) : r2(make_float2(q.r, q.r)) {}
-  __device__ __forceinline__ float2 operator()(float2 x) const { return __fmul2_rn(x, r2); }
+  float2 nr2;
+  __device__ __forceinline__ explicit PairExact(const Quotient& q) : nr2(make_float2(-q.r, -q.r)) {}
+  __device__ __forceinline__ float2 operator()(float2 nx) const { return __fmul2_rn(nx, nr2); }
 };
 struct PairCorrected {          // Markstein's correction with the rounded reciprocal
-  float2 r2, ns2;
+  float2 nr2, s2;
   __device__ __forceinline__ explicit PairCorrected(const Quotient& q)
-      : r2(make_float2(q.r, q.r)), ns2(make_float2(-q.s, -q.s)) {}
-  __device__ __forceinline__ float2 operator()(float2 x) const {
-    const float2 q0 = __fmul2_rn(x, r2);
-    const float2 e = __ffma2_rn(q0, ns2, x);    // x - q0 s, exact
-    const float2 y = __ffma2_rn(e, r2, q0);
-    return make_float2(copysignf(y.x, x.x), copysignf(y.y, x.y));
+      : nr2(make_float2(-q.r, -q.r)), s2(make_float2(q.s, q.s)) {}
+  __device__ __forceinline__ float2 operator()(float2 nx) const {
+    const float2 q0 = __fmul2_rn(nx, nr2);      // RN(x r)
+    const float2 d = __ffma2_rn(q0, s2, nx);    // q0 s - x, exact
+    return __ffma2_rn(d, nr2, q0);              // RN(q0 - d r)
   }
 };
 struct PairGeneral {            // any rule, decided per call
   Quotient q;
   __device__ __forceinline__ explicit PairGeneral(const Quotient& q_) : q(q_) {}
-  __device__ __forceinline__ float2 operator()(float2 x) const { return make_float2(q(x.x), q(x.y)); }
+  __device__ __forceinline__ float2 operator()(float2 nx) const { return make_float2(q(-nx.x), q(-nx.y)); }
 };
 
 // Runs body(pair quotient of the calling lane's tile) with the rule picked once per warp.
@@ -365,10 +375,10 @@ __global__ void __launch_bounds__(256, 6) quant_act_dual_kernel(const __grid_con
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const uint4 w = v[j];
-        const float2 p0 = qd(make_float2(bf16lo(w.x), bf16hi(w.x)));
-        const float2 p1 = qd(make_float2(bf16lo(w.y), bf16hi(w.y)));
-        const float2 p2 = qd(make_float2(bf16lo(w.z), bf16hi(w.z)));
-        const float2 p3 = qd(make_float2(bf16lo(w.w), bf16hi(w.w)));
+        const float2 p0 = qd(make_float2(bf16lo_neg(w.x), bf16hi_neg(w.x)));
+        const float2 p1 = qd(make_float2(bf16lo_neg(w.y), bf16hi_neg(w.y)));
+        const float2 p2 = qd(make_float2(bf16lo_neg(w.z), bf16hi_neg(w.z)));
+        const float2 p3 = qd(make_float2(bf16lo_neg(w.w), bf16hi_neg(w.w)));
         uint2 o;
         o.x = __byte_perm(cvt_e4m3x2(p0.x, p0.y), cvt_e4m3x2(p1.x, p1.y), 0x5410);
         o.y = __byte_perm(cvt_e4m3x2(p2.x, p2.y), cvt_e4m3x2(p3.x, p3.y), 0x5410);
@@ -402,8 +412,8 @@ __global__ void __launch_bounds__(256, 6) quant_act_dual_kernel(const __grid_con
     with_pair_quotient(Quotient(sc), [&](const auto& qd) {
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        const float2 e0 = qd(make_float2(bf16lo(w2[2 * c]), bf16hi(w2[2 * c])));
-        const float2 e1 = qd(make_float2(bf16lo(w2[2 * c + 1]), bf16hi(w2[2 * c + 1])));
+        const float2 e0 = qd(make_float2(bf16lo_neg(w2[2 * c]), bf16hi_neg(w2[2 * c])));
+        const float2 e1 = qd(make_float2(bf16lo_neg(w2[2 * c + 1]), bf16hi_neg(w2[2 * c + 1])));
         vv[c] = __byte_perm(cvt_e4m3x2(e0.x, e0.y), cvt_e4m3x2(e1.x, e1.y), 0x5410);
       }
     });

@@ -4,7 +4,10 @@
  * The kernels compute x / s without a division for most tiles (see Quotient in
  * fp8_fine_grained_weight_b200/csrc/quant.cuh): a power-of-two s uses the exact
  * reciprocal; s >= 2^-92 uses a correctly rounded reciprocal plus one FMA residual
- * correction; smaller s divide.  This program replays that sequence with IEEE
+ * correction, with the residual taken as d = q0 s - x and the quotient as RN(q0 - d r)
+ * so that x = -0 keeps its sign without a sign restore (the f32x2 path feeds the
+ * negated input -x and -r, the same values); smaller s divide.  This program replays
+ * that sequence with IEEE
  * single-precision host arithmetic (the GPU's fmul/fma/rcp.rn are IEEE too) for
  * every positive finite bf16 amax, both scale modes, and every bf16 x with
  * |x| <= amax, and checks that it yields the same E4M3 input as RN(x / s):
@@ -81,12 +84,13 @@ int main(void) {
                     float x = f_of(((uint32_t)xb << 16) | (sg ? 0x80000000u : 0));
                     float ref = x / s;
                     float q;
+                    const float nx = -x, nr = -r;   /* the f32x2 path's operands */
                     if (mode == 0) {
-                        q = x * r;
+                        q = nx * nr;
                     } else {
-                        float q0 = x * r;
-                        float e = fmaf(-q0, s, x);
-                        q = copysignf(fmaf(e, r, q0), x);
+                        float q0 = nx * nr;
+                        float d = fmaf(q0, s, nx);
+                        q = fmaf(d, nr, q0);
                     }
                     ++checked;
                     if (fabsf(ref) >= 0x1p-11f) {
