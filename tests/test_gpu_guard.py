@@ -140,10 +140,13 @@ def test_gemm_blockscaled_guard(fq, M, N, K, out_fp32):
     C.check(f"gemm_blockscaled {M}x{N}x{K}")
 
 
+# M = 300: CTA-pair tiles of 256 rows (the second pair's odd CTA has no rows); M = 77:
+# one-CTA tiles of 128 rows.
+@pytest.mark.parametrize("M", [300, 77])
 @pytest.mark.parametrize("rowwise", [False, True])
-def test_gemm_ue8m0_and_nopromo_guard(fq, rowwise):
+def test_gemm_ue8m0_and_nopromo_guard(fq, rowwise, M):
     import torch
-    M, N, K = 300, 640, 512            # 640 = 2.86 tiles of 224 columns: a partial last tile
+    N, K = 640, 512                    # 640 = 2.86 tiles of 224 columns: a partial last tile
     qa, sa, qb, sb = _gemm_operands(fq, M, N, K, 11, pow2=True, rowwise=rowwise)
     C = Guarded(M, N, N + 32, torch.bfloat16)
     fq.gemm_blockscaled_ue8m0(qa, sa, qb, sb, b_rowwise=rowwise, out=C.view)
