@@ -208,72 +208,34 @@ int64_t dense_tiles(int64_t M, int64_t N) {
 
 static_assert(fp8q::kErrScale == FP8Q_ERR_SCALE, "device status code of a bad scale");
 
-// Launch of the power-of-two-scale GEMM: one persistent CTA (PAIR: CTA pair, launched as
-// clusters of 2) per SM or SM pair; kernel attributes set and the co-resident count
-// cached per device on first use.  work: tiles (a bound for grouped).
-template <bool ROW_B, bool OUT_BF16, bool GROUPED, bool PAIR>
+// Launch of the power-of-two-scale GEMM: one persistent CTA per SM (kernel attributes set
+// and the co-resident count cached per device on first use).  work: tiles (a bound for
+// grouped).
+template <bool ROW_B, bool OUT_BF16, bool GROUPED>
 int run_gemm_ue8m0(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
                    int64_t work, cudaStream_t st) {
-  using Cfg = fp8q::Ue8m0Cfg<GROUPED, PAIR>;
-  static constexpr auto kern = fp8q::gemm_fp8_ue8m0_kernel<ROW_B, OUT_BF16, GROUPED, PAIR>;
+  using Cfg = fp8q::Ue8m0Cfg<GROUPED>;
+  static constexpr auto kern = fp8q::gemm_fp8_ue8m0_kernel<ROW_B, OUT_BF16, GROUPED>;
   static std::atomic<int> cached[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8Q_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = Cfg::kCG;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(Cfg::kThreads);
-  cfg.dynamicSmemBytes = Cfg::smem_bytes;
-  cfg.stream = st;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int units = cached[dev].load(std::memory_order_acquire);   // co-resident tiles (MMA units)
+  int units = cached[dev].load(std::memory_order_acquire);
   if (units == 0) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(Cfg::smem_bytes)) != cudaSuccess)
       return FP8Q_ERR_CUDA;
-    if (PAIR) {
-      int clusters = 0;
-      cfg.gridDim = dim3(2 * Cfg::kCG);
-      if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters <= 0)
-        return FP8Q_ERR_CUDA;
-      units = clusters;
-    } else {
-      int sms = 0, per_sm = 0;
-      if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Cfg::kThreads, Cfg::smem_bytes) !=
-              cudaSuccess || per_sm <= 0)
-        return FP8Q_ERR_CUDA;
-      units = sms * per_sm;
-    }
+    int sms = 0, per_sm = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Cfg::kThreads, Cfg::smem_bytes) !=
+            cudaSuccess || per_sm <= 0)
+      return FP8Q_ERR_CUDA;
+    units = sms * per_sm;
     cached[dev].store(units, std::memory_order_release);
   }
   const int64_t grid = work < units ? work : units;
   if (grid <= 0) return FP8Q_OK;
-  cfg.gridDim = dim3(static_cast<unsigned>(grid * Cfg::kCG));
-  if (cudaLaunchKernelEx(&cfg, kern, tmA, tmB, a) != cudaSuccess) return FP8Q_ERR_CUDA;
+  kern<<<static_cast<unsigned>(grid), Cfg::kThreads, Cfg::smem_bytes, st>>>(tmA, tmB, a);
   return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
-}
-
-// Dense power-of-two-scale GEMM: CTA pairs (256-row tiles) once M spans two row tiles.
-template <bool PAIR>
-int launch_dense_ue8m0(const uint8_t* A, const uint8_t* B, int64_t K, int64_t lda, int64_t ldb,
-                       const GemmArgs& a, bool row_b, bool bf16, cudaStream_t s) {
-  using Cfg = fp8q::Ue8m0Cfg<false, PAIR>;
-  CUtensorMap tmA, tmB;
-  int st;
-  if ((st = encode_operand(&tmA, A, K, a.M, lda, 128)) != FP8Q_OK) return st;
-  if ((st = encode_operand(&tmB, B, K, a.N, ldb, Cfg::kBRows)) != FP8Q_OK) return st;
-  const int64_t tiles = ((a.M + Cfg::kTileM - 1) / Cfg::kTileM) * ((a.N + Cfg::kN - 1) / Cfg::kN);
-  if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  if (bf16)
-    return row_b ? run_gemm_ue8m0<true, true, false, PAIR>(tmA, tmB, a, tiles, s)
-                 : run_gemm_ue8m0<false, true, false, PAIR>(tmA, tmB, a, tiles, s);
-  return row_b ? run_gemm_ue8m0<true, false, false, PAIR>(tmA, tmB, a, tiles, s)
-               : run_gemm_ue8m0<false, false, false, PAIR>(tmA, tmB, a, tiles, s);
 }
 
 }  // namespace
@@ -514,17 +476,26 @@ int fp8_gemm_blockscaled_ue8m0(const uint8_t* A, const float* sA, int64_t ld_sa,
                                const uint8_t* B, const float* sB, int64_t ld_sb, int b_scale_mode,
                                void* C, int out_dtype, int64_t M, int64_t N, int64_t K,
                                int64_t lda, int64_t ldb, int64_t ldc, void* stream) {
+  using Cfg = fp8q::Ue8m0Cfg<false>;
   if (M == 0 && N >= 0 && K >= 0) return FP8Q_OK;
   int st = check_dense_blockscaled(A, sA, ld_sa, B, sB, ld_sb, b_scale_mode, C, out_dtype, M, N, K,
                                    lda, ldb, ldc);
   if (st != FP8Q_OK) return st;
+  CUtensorMap tmA, tmB;
+  if ((st = encode_operand(&tmA, A, K, M, lda, Cfg::kTileM)) != FP8Q_OK) return st;
+  if ((st = encode_operand(&tmB, B, K, N, ldb, Cfg::kN)) != FP8Q_OK) return st;
   GemmArgs a{};
   a.sA = sA; a.ld_sa = ld_sa; a.sB = sB; a.ld_sb = ld_sb; a.C = C; a.ldc = ldc;
   a.M = M; a.N = N; a.G = static_cast<int>(K / 128); a.m_offsets = nullptr; a.num_experts = 0;
+  const int64_t tiles = ((M + Cfg::kTileM - 1) / Cfg::kTileM) * ((N + Cfg::kN - 1) / Cfg::kN);
+  if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   const auto s = static_cast<cudaStream_t>(stream);
-  const bool row_b = b_scale_mode == FP8Q_BSCALE_ROW1x128, bf16 = out_dtype == FP8Q_OUT_BF16;
-  return M > 128 ? launch_dense_ue8m0<true>(A, B, K, lda, ldb, a, row_b, bf16, s)
-                 : launch_dense_ue8m0<false>(A, B, K, lda, ldb, a, row_b, bf16, s);
+  const bool row_b = b_scale_mode == FP8Q_BSCALE_ROW1x128;
+  if (out_dtype == FP8Q_OUT_BF16)
+    return row_b ? run_gemm_ue8m0<true, true, false>(tmA, tmB, a, tiles, s)
+                 : run_gemm_ue8m0<false, true, false>(tmA, tmB, a, tiles, s);
+  return row_b ? run_gemm_ue8m0<true, false, false>(tmA, tmB, a, tiles, s)
+               : run_gemm_ue8m0<false, false, false>(tmA, tmB, a, tiles, s);
 }
 
 int fp8_gemm_grouped_ue8m0(const uint8_t* A, const float* sA, int64_t ld_sa, const uint8_t* W,
@@ -553,8 +524,8 @@ int fp8_gemm_grouped_ue8m0(const uint8_t* A, const float* sA, int64_t ld_sa, con
                         ((N + Cfg::kN - 1) / Cfg::kN);
   if (bound > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   const auto s = static_cast<cudaStream_t>(stream);
-  return out_dtype == FP8Q_OUT_BF16 ? run_gemm_ue8m0<false, true, true, false>(tmA, tmB, a, bound, s)
-                                    : run_gemm_ue8m0<false, false, true, false>(tmA, tmB, a, bound, s);
+  return out_dtype == FP8Q_OUT_BF16 ? run_gemm_ue8m0<false, true, true>(tmA, tmB, a, bound, s)
+                                    : run_gemm_ue8m0<false, false, true>(tmA, tmB, a, bound, s);
 }
 
 int fp8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, size_t* bytes) {

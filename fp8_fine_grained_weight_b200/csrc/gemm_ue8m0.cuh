@@ -17,35 +17,28 @@
 // (kSiteScaleFormat << 8) | FP8Q_ERR_SCALE in the device error word for them and goes on
 // with scale 1.
 //
-// PAIR = false: tiles of 128 x 224, one CTA each.  PAIR = true: tiles of 256 x 224 on a
-// CTA pair (cluster of 2, tcgen05 cta_group::2): CTA r loads A rows 128 r.. and B rows
-// 112 r.. of the tile (30 KB per stage instead of 44 KB, so 7 stages), the even CTA
-// issues the M = 256 MMAs and the scale copies (tcgen05.cp.cta_group::2: each CTA's
-// shared memory into its own TMEM), and its commits arrive on both CTAs' barriers; the
-// odd CTA's producers and epilogue signal the even CTA's barriers remotely.  No TMA
-// multicast.  224 columns: two 224-column FP32 accumulators and the scale region fill
-// the 512 TMEM columns, and 224 divides 7168.  GROUPED: the MoE form of fp8_gemm_grouped
-// -- tiles come from a per-expert table built from m_offsets on the device (n fastest
-// inside an expert), A rows past an expert's end are masked, B rows come from the stacked
-// expert weights with that expert's block scales, and the ring has fewer stages to leave
-// room for the table.
-//   warp 0       TMA producer: A [128 x 128 B] and this CTA's B rows [224 or 112 x 128 B]
-//                per K-group into the stage ring (128-byte swizzle).
-//   warp 1       TMEM owner; in the MMA-issuing CTA also the MMA issuer.  Per slot of four
-//                groups it copies the slot's scale words from shared memory into TMEM
-//                (tcgen05.cp 32x128b.warpx4: a 32-row x 16-byte block into 4 columns of
-//                every 32-lane sub-partition), then issues the groups' block-scaled MMAs
-//                (K = 32 each).  tcgen05.cp and tcgen05.mma of one thread run in issue
-//                order, so a scale slot in TMEM is rewritten only after the MMAs that read
-//                it.  Commits free smem stages, scale slots and finished accumulators.
+// Tiles of 128 x 224 (224 divides 7168; two 224-column FP32 accumulators and the scale
+// region fill the 512 TMEM columns), persistent CTAs, 12 warps.  GROUPED: the MoE form of
+// fp8_gemm_grouped -- tiles come from a per-expert table built from m_offsets on the
+// device (n fastest inside an expert), A rows past an expert's end are masked, B rows
+// come from the stacked expert weights with that expert's block scales, and the ring has
+// 4 stages to leave room for the table.
+//   warp 0       TMA producer: A [128 x 128 B] and B [224 x 128 B] per K-group into a
+//                5-stage ring (4 when grouped; 128-byte swizzle).
+//   warp 1       TMEM owner and MMA issuer.  Per slot of four groups it copies the slot's
+//                scale words from shared memory into TMEM (tcgen05.cp 32x128b.warpx4: a
+//                32-row x 16-byte block into 4 columns of every 32-lane sub-partition),
+//                then issues the groups' block-scaled MMAs (K = 32 each).  tcgen05.cp and
+//                tcgen05.mma of one thread run in issue order, so a scale slot in TMEM is
+//                rewritten only after the MMAs that read it.  Commits free smem stages,
+//                scale slots and finished accumulators.
 //   warp 2       scale producer.  For a slot (groups 4k .. 4k+3 of one tile) lane l packs
 //                the UE8M0 bytes of A rows l, 32+l, 64+l, 96+l (byte j = group 4k+j) into
-//                one 16-byte row of the A block, and those of B rows l + 32j into two
-//                16-byte rows of the B blocks, in a 3-slot shared-memory ring.  After the
-//                copies the MMA reads, for A row m, lane m and column m/32, and for B row
-//                n, column 4 + n/32 and lane n % 32 of its own sub-partition: the layout
-//                of kind::mxf8f6f4 scale factors (checked on B200 with probes; for the
-//                pair, which B rows each CTA's blocks carry is kSfbSplit).
+//                one 16-byte row of the A block, and those of B rows l + 32j (j < 7) into
+//                two 16-byte rows of the B blocks, in a 3-slot shared-memory ring.  After
+//                the copies the MMA reads, for A row m, lane m and column m/32, and for B
+//                row n, column 4 + n/32 and lane n % 32 of its own sub-partition: the
+//                layout of kind::mxf8f6f4 scale factors (checked on B200 with probes).
 //   warp 3       idle.
 //   warps 4-11   epilogue: warp w drains TMEM lanes 32*(w%4).. and 112 of the 224
 //                columns of a finished accumulator, converts and stores C, and frees the
@@ -62,13 +55,11 @@ namespace fp8q {
 constexpr unsigned int kSiteScaleFormat = 8;
 constexpr unsigned int kErrScale = 7;            // FP8Q_ERR_SCALE
 
-template <bool GROUPED, bool PAIR = false>
+template <bool GROUPED>
 struct Ue8m0Cfg {
-  static constexpr int kCG = PAIR ? 2 : 1;        // CTAs per MMA
-  static constexpr int kTileM = 128 * kCG;
+  static constexpr int kTileM = 128;
   static constexpr int kN = 224;                  // tile columns = MMA N
-  static constexpr int kBRows = kN / kCG;         // B rows each CTA loads per stage
-  static constexpr int kStages = PAIR ? (GROUPED ? 6 : 7) : (GROUPED ? 4 : 5);
+  static constexpr int kStages = GROUPED ? 4 : 5; // grouped: room for the tile table
   static constexpr int kAccCols = 2 * kN;         // two accumulator buffers
   static constexpr int kSfSmemSlots = 3;          // scale slots in shared memory, 4 groups each
   static constexpr int kSfTmemSlots = 4;          // scale slots in TMEM
@@ -78,15 +69,8 @@ struct Ue8m0Cfg {
   static constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
   static constexpr int kSetCols = kN / 2;         // columns per epilogue warp
   static constexpr uint32_t kABytes = 128 * kBK;
-  static constexpr uint32_t kBBytes = kBRows * kBK;
-  static constexpr uint32_t kStageTx = (kABytes + kBBytes) * kCG;   // bytes per full phase
-  // B rows whose scales a CTA's blocks carry: its own B rows (split) or the tile's all.
-  static constexpr bool kSfbSplit = false;
-  static constexpr int kSfbRows = (PAIR && kSfbSplit) ? kBRows : kN;
-  static constexpr int kSfbChunks = (kSfbRows + 31) / 32;
-  // accumulator release: every epilogue thread (one CTA), one remote arrive per epilogue
-  // warp of both CTAs (pair)
-  static constexpr uint32_t kTemptyArrivals = PAIR ? kCG * kEpiWarps : 32 * kEpiWarps;
+  static constexpr uint32_t kBBytes = kN * kBK;
+  static constexpr uint32_t kStageTx = kABytes + kBBytes;
   static constexpr uint32_t kSfA = 32 * 16;       // one 32 x 16 B copy block
   static constexpr uint32_t kSfBytes = 3 * kSfA;  // A block, two B blocks
   static constexpr uint32_t a = 0;
@@ -100,8 +84,8 @@ struct Ue8m0Cfg {
   static constexpr uint32_t end = sched + (GROUPED ? 4 * (kMaxGroups + 1) : 0);
   static constexpr uint32_t smem_bytes = end + 1024;
   static_assert(kAccCols + kSfTmemSlots * kSfSlotCols <= static_cast<int>(kTmemCols), "TMEM budget");
-  static_assert(kSfbChunks <= 8, "B scales fit two copy blocks");
-  static_assert(kN % 16 == 0 && kN <= 256, "MMA N");
+  static_assert((kN + 31) / 32 <= 8, "B scales fit two copy blocks");
+  static_assert(kN % 16 == 0 && kN <= 256, "MMA N for M = 128");
   static_assert(kSetCols % 16 == 0, "16-column epilogue loads");
   static_assert(kABytes % 1024 == 0 && kBBytes % 1024 == 0 && sf % 1024 == 0, "alignment");
   static_assert(smem_bytes <= 232448, "fits the 227 KB opt-in shared memory");
@@ -118,13 +102,8 @@ __device__ __forceinline__ uint64_t smem_desc_copy32x16(uint32_t saddr) {
   return d;
 }
 
-// CG = 2: issued by the even CTA, each CTA's shared memory into its own TMEM.
-template <int CG>
 __device__ __forceinline__ void tmem_copy_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
-  if (CG == 1)
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-  else
-    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -141,13 +120,12 @@ __device__ __forceinline__ uint32_t ue8m0_of(float s, bool& bad) {
   return 127;
 }
 
-template <bool ROW_B, bool OUT_BF16, bool GROUPED, bool PAIR>
-__global__ void __launch_bounds__(Ue8m0Cfg<GROUPED, PAIR>::kThreads, 1)
+template <bool ROW_B, bool OUT_BF16, bool GROUPED>
+__global__ void __launch_bounds__(Ue8m0Cfg<GROUPED>::kThreads, 1)
     gemm_fp8_ue8m0_kernel(const __grid_constant__ CUtensorMap tmA,
                           const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
-  using Cfg = Ue8m0Cfg<GROUPED, PAIR>;
+  using Cfg = Ue8m0Cfg<GROUPED>;
   static_assert(!(GROUPED && ROW_B), "grouped GEMMs take 128x128 weight-block scales");
-  constexpr int CG = Cfg::kCG;
   constexpr int S = Cfg::kStages;
   constexpr int SF = Cfg::kSfSmemSlots;
   constexpr int TS = Cfg::kSfTmemSlots;
@@ -169,13 +147,6 @@ __global__ void __launch_bounds__(Ue8m0Cfg<GROUPED, PAIR>::kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.G;
-  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;   // CTA 0 of a pair issues the MMAs
-  const bool mma_cta = rank == 0;
-  const int unit0 = blockIdx.x / CG, units = gridDim.x / CG;   // cluster index / count
-  // a commit that frees or publishes something both CTAs of a pair wait for
-  auto commit_all = [&](uint32_t bar) {
-    if (PAIR) mma_commit_pair(bar, 0x3); else mma_commit<1>(bar);
-  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -184,10 +155,10 @@ __global__ void __launch_bounds__(Ue8m0Cfg<GROUPED, PAIR>::kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), Cfg::kTemptyArrivals);
+      mbar_init(tempty_bar(b), 32 * Cfg::kEpiWarps);   // every epilogue thread
     }
     for (int r = 0; r < SF; ++r) {
-      mbar_init(sfull_bar(r), CG);                      // each CTA's scale producer
+      mbar_init(sfull_bar(r), 1);                       // the scale producer
       mbar_init(sempty_bar(r), 1);                      // the MMA thread's commit
     }
     mbar_init(drain_bar, 1);
@@ -199,8 +170,8 @@ __global__ void __launch_bounds__(Ue8m0Cfg<GROUPED, PAIR>::kThreads, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc<CG>(smem_u32(tmem_slot), kTmemCols);
-    tmem_relinquish<CG>();
+    tmem_alloc<1>(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish<1>();
   }
   const int nt_total = static_cast<int>((p.N + kN - 1) / kN);
   int* sched = reinterpret_cast<int*>(smem + Cfg::sched);
@@ -224,15 +195,14 @@ __global__ void __launch_bounds__(Ue8m0Cfg<GROUPED, PAIR>::kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (PAIR) cluster_sync();       // the peer's barriers are initialised before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   if (GROUPED) num_tiles = sched[p.num_experts];
-  // Tiles of this CTA (pair): unit0, + units, ...; dense: m-fastest so that the units of a
-  // wave share B tiles; grouped: expert by expert, n-fastest inside an expert.
-  const int n_tiles = unit0 < num_tiles ? (num_tiles - unit0 + units - 1) / units : 0;
+  // Tiles of this CTA: blockIdx.x, + gridDim.x, ...; dense: m-fastest so that the CTAs
+  // of a wave share B tiles; grouped: expert by expert, n-fastest inside an expert.
+  const int n_tiles = blockIdx.x < num_tiles ? (num_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
   auto tile_of = [&](int i) -> Tile {
-    return decode_tile<GROUPED, Cfg::kTileM, kN>(unit0 + i * units, p, mt_total, nt_total, sched);
+    return decode_tile<GROUPED, Cfg::kTileM, kN>(blockIdx.x + i * gridDim.x, p, mt_total, nt_total, sched);
   };
 
   if (warp == 0) {
@@ -242,39 +212,26 @@ __global__ void __launch_bounds__(Ue8m0Cfg<GROUPED, PAIR>::kThreads, 1)
       bool ok = true;
       for (int i = 0; ok && i < n_tiles; ++i) {
         const Tile tl = tile_of(i);
-        const int32_t arow = static_cast<int32_t>(tl.row0 + 128 * rank);
-        const int32_t brow = static_cast<int32_t>(tl.brow0 + Cfg::kBRows * rank);
         for (int g = 0; g < G; ++g, ++it) {
           const int s = it % S;
           if (!mbar_wait(empty_bar(s), ((it / S) & 1u) ^ 1u, kSiteProducer, abort_flag)) {
             ok = false;
             break;
           }
-          if (mma_cta) mbar_arrive_expect_tx(full_bar(s), Cfg::kStageTx);
-          const uint32_t dst_a = sbase + Cfg::a + s * Cfg::kABytes;
-          const uint32_t dst_b = sbase + Cfg::b + s * Cfg::kBBytes;
-          if (PAIR) {
-            const uint32_t fb = map_shared_rank(full_bar(s), 0);   // the MMA CTA's barrier
-            tma_load_2d_pair(dst_a, &tmA, fb, g * kBK, arow);
-            tma_load_2d_pair(dst_b, &tmB, fb, g * kBK, brow);
-          } else {
-            tma_load_2d(dst_a, &tmA, full_bar(s), g * kBK, arow);
-            tma_load_2d(dst_b, &tmB, full_bar(s), g * kBK, brow);
-          }
+          mbar_arrive_expect_tx(full_bar(s), Cfg::kStageTx);
+          tma_load_2d(sbase + Cfg::a + s * Cfg::kABytes, &tmA, full_bar(s), g * kBK,
+                      static_cast<int32_t>(tl.row0));
+          tma_load_2d(sbase + Cfg::b + s * Cfg::kBBytes, &tmB, full_bar(s), g * kBK,
+                      static_cast<int32_t>(tl.brow0));
         }
       }
-      // Every issued load lands before the CTA can exit.  The MMA CTA watches its full
-      // barriers (bounded; loads finish on their own); the other CTA's loads complete on
-      // the MMA CTA's barriers and were consumed before the final cluster barrier (after
-      // an abort the teardown waits a fixed while).
-      if (mma_cta) {
-        const uint32_t first = it > static_cast<uint32_t>(S) ? it - S : 0;
-        for (uint32_t j = first; j < it; ++j) mbar_wait(full_bar(j % S), (j / S) & 1u, kSiteDrain, nullptr);
-      }
+      // every issued load lands before the CTA can exit (bounded; loads end on their own)
+      const uint32_t first = it > static_cast<uint32_t>(S) ? it - S : 0;
+      for (uint32_t j = first; j < it; ++j) mbar_wait(full_bar(j % S), (j / S) & 1u, kSiteDrain, nullptr);
     }
   } else if (warp == 1) {
     // -------------------------------------------------------------- MMA issuer
-    if (lane == 0 && mma_cta) {
+    if (lane == 0) {
       uint32_t it = 0, sc = 0;     // groups and scale slots issued so far
       bool ok = true;
       for (int i = 0; ok && i < n_tiles; ++i) {
@@ -286,15 +243,15 @@ __global__ void __launch_bounds__(Ue8m0Cfg<GROUPED, PAIR>::kThreads, 1)
           const int r = sc % SF;
           const uint32_t sfa = tmem_base + Cfg::kSfCol0 + (sc % TS) * Cfg::kSfSlotCols;
           if ((g & 3) == 0) {
-            if (!mbar_wait<PAIR>(sfull_bar(r), (sc / SF) & 1u, kSiteScales, abort_flag)) {
+            if (!mbar_wait(sfull_bar(r), (sc / SF) & 1u, kSiteScales, abort_flag)) {
               ok = false;
               break;
             }
             tc_fence_after();
             const uint32_t src = sbase + Cfg::sf + r * Cfg::kSfBytes;
-            tmem_copy_32x128b_x4<CG>(sfa, smem_desc_copy32x16(src));
-            tmem_copy_32x128b_x4<CG>(sfa + 4, smem_desc_copy32x16(src + Cfg::kSfA));
-            tmem_copy_32x128b_x4<CG>(sfa + 8, smem_desc_copy32x16(src + 2 * Cfg::kSfA));
+            tmem_copy_32x128b_x4(sfa, smem_desc_copy32x16(src));
+            tmem_copy_32x128b_x4(sfa + 4, smem_desc_copy32x16(src + Cfg::kSfA));
+            tmem_copy_32x128b_x4(sfa + 8, smem_desc_copy32x16(src + 2 * Cfg::kSfA));
           }
           if (!mbar_wait(full_bar(s), (it / S) & 1u, kSiteMmaFull, abort_flag)) {
             ok = false;
@@ -308,18 +265,18 @@ __global__ void __launch_bounds__(Ue8m0Cfg<GROUPED, PAIR>::kThreads, 1)
           const uint32_t b_addr = sbase + Cfg::b + s * Cfg::kBBytes;
 #pragma unroll
           for (int kk = 0; kk < kBK / 32; ++kk)
-            mma_f8_ue8m0<CG>(d, smem_desc_k_sw128(a_addr + 32 * kk), smem_desc_k_sw128(b_addr + 32 * kk),
-                             idesc, (g > 0 || kk > 0) ? 1u : 0u, sfa_b, sfb_b);
-          commit_all(empty_bar(s));
+            mma_f8_ue8m0(d, smem_desc_k_sw128(a_addr + 32 * kk), smem_desc_k_sw128(b_addr + 32 * kk),
+                         idesc, (g > 0 || kk > 0) ? 1u : 0u, sfa_b, sfb_b);
+          mma_commit<1>(empty_bar(s));
           if ((g & 3) == 3 || g == G - 1) {       // the slot's last group: free it when read
-            commit_all(sempty_bar(r));
+            mma_commit<1>(sempty_bar(r));
             ++sc;
           }
         }
         if (!ok) break;
-        commit_all(tfull_bar(buf));
+        mma_commit<1>(tfull_bar(buf));
       }
-      mma_commit<CG>(drain_bar);
+      mma_commit<1>(drain_bar);
       mbar_wait(drain_bar, 0, kSiteDrain, nullptr);
     }
   } else if (warp == Cfg::kSfWarp) {
@@ -327,50 +284,54 @@ __global__ void __launch_bounds__(Ue8m0Cfg<GROUPED, PAIR>::kThreads, 1)
     // Slots hold four groups of one tile (4k .. 4k + 3; a tile's last slot may be
     // partial); the CTA's slots run in order (tile i, slot k), and the raw scales of the
     // next slot are loaded before the current one is stored.
-    //   A: lane l loads the 4 groups' scales of this CTA's rows l + 32j, j < 4.
-    //   B: lane l loads the 4 groups' scales of B rows n = bbase + l + 32j, j < kSfbChunks
-    //     (128x128 blocks: the scale of block n / 128; 1x128 rows: the row's own scale).
-    constexpr int kChB = Cfg::kSfbChunks;
+    //   A: lane l loads the 4 groups' scales of rows l + 32j, j < 4.
+    //   B, 128x128 blocks: the tile's 224 rows touch at most 3 blocks; lane l < 12 loads
+    //     block nb0 + l / 4, group 4k + l % 4, and shuffles build the packed words (every
+    //     32-row chunk of the tile lies inside one block).
+    //   B, 1x128 rows: lane l loads the 4 groups' scales of rows l + 32j, j < 7.
+    constexpr int kRawB = ROW_B ? 28 : 1;
     struct Raw {
       float a[16];
-      float b[4 * kChB];
+      float b[kRawB];
     };
     bool bad = false;
     auto fetch = [&](int i, int k, Raw& raw) {
 #pragma unroll
       for (int j = 0; j < 16; ++j) raw.a[j] = 1.0f;
 #pragma unroll
-      for (int j = 0; j < 4 * kChB; ++j) raw.b[j] = 1.0f;
+      for (int j = 0; j < kRawB; ++j) raw.b[j] = 1.0f;
       if (i >= n_tiles) return;
       const Tile tl = tile_of(i);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int64_t m = tl.row0 + 128 * rank + 32 * j + lane;
+        const int64_t m = tl.row0 + 32 * j + lane;
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
           const int g = 4 * k + b;
           if (g < G && m < tl.row_end) raw.a[4 * j + b] = __ldg(p.sA + static_cast<int64_t>(g) * p.ld_sa + m);
         }
       }
-      const int64_t bbase = tl.col0 + (Cfg::kSfbRows < kN ? Cfg::kBRows * rank : 0);
-      const int64_t bend = bbase + Cfg::kSfbRows;           // this CTA's B rows of the tile
+      if (ROW_B) {
 #pragma unroll
-      for (int j = 0; j < kChB; ++j) {
-        const int64_t n = bbase + 32 * j + lane;
-        const bool nv = n < bend && n < p.N;
+        for (int j = 0; j < 7; ++j) {
+          const int64_t n = tl.col0 + 32 * j + lane;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const int g = 4 * k + b;
-          if (g < G && nv) {
-            raw.b[4 * j + b] = ROW_B ? __ldg(p.sB + static_cast<int64_t>(g) * p.ld_sb + n)
-                                     : __ldg(p.sB + (static_cast<int64_t>(tl.expert) * (p.N / 128) + n / 128) * G + g);
+          for (int b = 0; b < 4; ++b) {
+            const int g = 4 * k + b;
+            if (g < G && n < p.N) raw.b[4 * j + b] = __ldg(p.sB + static_cast<int64_t>(g) * p.ld_sb + n);
           }
         }
+      } else {
+        const int64_t nb = tl.col0 / 128 + (lane >> 2);
+        const int g = 4 * k + (lane & 3);
+        if (lane < 12 && g < G && nb * 128 < p.N)
+          raw.b[0] = __ldg(p.sB + (static_cast<int64_t>(tl.expert) * (p.N / 128) + nb) * G + g);
       }
     };
     // Packs the slot into its shared-memory blocks once the MMA thread has copied the
     // ring slot's previous contents.  Returns false (warp-uniform) on abort or timeout.
-    auto emit = [&](int64_t sc, const Raw& raw) -> bool {
+    auto emit = [&](int i, int64_t sc, const Raw& raw) -> bool {
+      const Tile tl = tile_of(i);
       uint32_t wa[4], wb[8];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -378,14 +339,30 @@ __global__ void __launch_bounds__(Ue8m0Cfg<GROUPED, PAIR>::kThreads, 1)
 #pragma unroll
         for (int b = 0; b < 4; ++b) wa[j] |= ue8m0_of(raw.a[4 * j + b], bad) << (8 * b);
       }
+      if (ROW_B) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        wb[j] = 0;
-        if (j < kChB) {
+        for (int j = 0; j < 7; ++j) {
+          wb[j] = 0;
 #pragma unroll
           for (int b = 0; b < 4; ++b) wb[j] |= ue8m0_of(raw.b[4 * j + b], bad) << (8 * b);
         }
+      } else {
+        const uint32_t byte = ue8m0_of(raw.b[0], bad);
+        uint32_t w[3];
+#pragma unroll
+        for (int jb = 0; jb < 3; ++jb) {
+          w[jb] = 0;
+#pragma unroll
+          for (int b = 0; b < 4; ++b) w[jb] |= __shfl_sync(0xFFFFFFFFu, byte, 4 * jb + b) << (8 * b);
+        }
+        const int nb0 = static_cast<int>(tl.col0 / 128);
+#pragma unroll
+        for (int j = 0; j < 7; ++j) {
+          const int jb = static_cast<int>((tl.col0 + 32 * j) / 128) - nb0;
+          wb[j] = jb == 0 ? w[0] : (jb == 1 ? w[1] : w[2]);
+        }
       }
+      wb[7] = 0;
       const int r = static_cast<int>(sc % SF);
       // warp-uniform outcome (the warp writes the slot together)
       const bool got = mbar_wait(sempty_bar(r), static_cast<uint32_t>(((sc / SF) & 1) ^ 1), kSiteScales,
@@ -397,10 +374,7 @@ __global__ void __launch_bounds__(Ue8m0Cfg<GROUPED, PAIR>::kThreads, 1)
       *reinterpret_cast<uint4*>(blk + 2 * Cfg::kSfA + 16 * lane) = make_uint4(wb[4], wb[5], wb[6], wb[7]);
       fence_proxy_async_smem();                          // visible to tcgen05.cp
       __syncwarp();
-      if (lane == 0) {
-        if (PAIR) mbar_arrive_cluster_release(map_shared_rank(sfull_bar(r), 0));
-        else mbar_arrive(sfull_bar(r));
-      }
+      if (lane == 0) mbar_arrive(sfull_bar(r));
       return true;
     };
     const int G4 = (G + 3) / 4;
@@ -410,7 +384,7 @@ __global__ void __launch_bounds__(Ue8m0Cfg<GROUPED, PAIR>::kThreads, 1)
     for (int i = 0, k = 0; i < n_tiles; ++sc) {
       const int i2 = k + 1 < G4 ? i : i + 1, k2 = k + 1 < G4 ? k + 1 : 0;
       fetch(i2, k2, nxt);
-      if (!emit(sc, cur)) break;
+      if (!emit(i, sc, cur)) break;
       cur = nxt;
       i = i2;
       k = k2;
@@ -429,7 +403,7 @@ __global__ void __launch_bounds__(Ue8m0Cfg<GROUPED, PAIR>::kThreads, 1)
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(tfull_bar(buf), (i >> 1) & 1u, kSiteEpilogue, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      const int64_t m = tl.row0 + 128 * rank + 32 * q + lane;
+      const int64_t m = tl.row0 + 32 * q + lane;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + buf * kN +
                              set * Cfg::kSetCols;
       const int64_t n_set = tl.col0 + set * Cfg::kSetCols;
@@ -460,37 +434,17 @@ __global__ void __launch_bounds__(Ue8m0Cfg<GROUPED, PAIR>::kThreads, 1)
         }
       }
       tc_fence_before();
-      if (PAIR) {                                        // accumulator free for tile i + 2
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(map_shared_rank(tempty_bar(buf), 0));
-      } else {
-        mbar_arrive(tempty_bar(buf));
-      }
+      mbar_arrive(tempty_bar(buf));                      // accumulator free for tile i + 2
     }
   }
 
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
-  if (PAIR) {
-    // After an abort the other CTA's in-flight loads into this CTA's shared memory are
-    // not tracked by any local barrier: give them a fixed, generous time to land.
-    if (*abort_flag) {
-      const uint64_t t0 = globaltimer();
-      while (globaltimer() - t0 < 200000ull) {
-      }
-    }
-    __syncwarp();
-    cluster_sync();
-  }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc<CG>(tmem_base, kTmemCols);
-  }
-  if (PAIR) {
-    __syncwarp();
-    cluster_sync();               // neither CTA exits while its peer may still address it
+    tmem_dealloc<1>(tmem_base, kTmemCols);
   }
 }
 

@@ -51,38 +51,26 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
-// CLUSTER: acquire at cluster scope, for phases that another CTA's release completes.
-template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
-  if (CLUSTER)
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.b32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-  else
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.b32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
   return ok != 0;
 }
 
 // Wait until the phase of parity `parity` has completed.  Returns false on timeout
 // (error recorded with `site`) or when `*abort` becomes nonzero.
-template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait_ns(uint32_t bar, uint32_t parity, unsigned int site,
                                              volatile int* abort, uint64_t timeout_ns) {
-  if (mbar_try_wait<CLUSTER>(bar, parity)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
-    if (mbar_try_wait<CLUSTER>(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     if (abort != nullptr && *abort) return false;
     if (globaltimer() - t0 > timeout_ns) {
       record_error((site << 8) | 6u /* FP8Q_ERR_TIMEOUT */);
@@ -92,10 +80,9 @@ __device__ __forceinline__ bool mbar_wait_ns(uint32_t bar, uint32_t parity, unsi
   }
 }
 
-template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned int site,
                                           volatile int* abort) {
-  return mbar_wait_ns<CLUSTER>(bar, parity, site, abort, FP8Q_WAIT_TIMEOUT_NS);
+  return mbar_wait_ns(bar, parity, site, abort, FP8Q_WAIT_TIMEOUT_NS);
 }
 
 // ---------------------------------------------------------------- TMA
@@ -170,13 +157,6 @@ __device__ __forceinline__ uint32_t map_shared_rank(uint32_t addr, uint32_t rank
 // shared-memory state, which CTA scope covers.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-
-// Same, releasing this thread's prior shared-memory writes to the cluster (the peer reads
-// them after its acquire).
-__device__ __forceinline__ void mbar_arrive_cluster_release(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
 }
 
 __device__ __forceinline__ void cluster_sync() {
@@ -361,26 +341,15 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_ue8m0(int M, int N, uint32_t s
 //   A scales: row m at lane m, column sfa + m / 32.
 //   B scales: row n at column sfb + n / 32, lane n % 32 of every 32-lane sub-partition
 //   (each sub-partition reads its own copy).
-// CG = 2: issued by the even CTA of a pair; every CTA reads the scales in its own TMEM
-// (its A rows' and, at the same columns, those of all N rows of B).
-template <int CG = 1>
 __device__ __forceinline__ void mma_f8_ue8m0(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                              uint32_t idesc, uint32_t accumulate, uint32_t sfa,
                                              uint32_t sfb) {
-  if (CG == 1)
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
-        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
-        : "memory");
-  else
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
-        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
-        : "memory");
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
 }
 
 // 16 consecutive TMEM columns of this warp's 32 lanes from / to registers.

@@ -168,8 +168,8 @@ int fp8_gemm_blockscaled(const uint8_t* A, const float* sA, int64_t ld_sa, const
  * differs).  Every scale the call reads must be a power of two in [2^-127, 2^127]; any
  * other value (not a power of two, zero, negative, inf, nan) is not detectable on the
  * host: the kernel records (8 << 8) | FP8Q_ERR_SCALE in the device error word, uses 1 in
- * its place and finishes the call (C is then not the product).  Tiles of 128 x 224 (one
- * CTA) for M <= 128, of 256 x 224 (a CTA pair) above; no workspace.
+ * its place and finishes the call (C is then not the product).  Tiles of 128 x 224; no
+ * workspace.
  */
 int fp8_gemm_blockscaled_ue8m0(const uint8_t* A, const float* sA, int64_t ld_sa,
                                const uint8_t* B, const float* sB, int64_t ld_sb, int b_scale_mode,

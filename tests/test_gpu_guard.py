@@ -140,8 +140,7 @@ def test_gemm_blockscaled_guard(fq, M, N, K, out_fp32):
     C.check(f"gemm_blockscaled {M}x{N}x{K}")
 
 
-# M = 300: CTA-pair tiles of 256 rows (the second pair's odd CTA has no rows); M = 77:
-# one-CTA tiles of 128 rows.
+# M = 300: three row tiles, the last one ragged; M = 77: one partial row tile.
 @pytest.mark.parametrize("M", [300, 77])
 @pytest.mark.parametrize("rowwise", [False, True])
 def test_gemm_ue8m0_and_nopromo_guard(fq, rowwise, M):
