@@ -459,6 +459,30 @@ def config_throughput(fq, flush_l2, reps=10):
                          "frac_of_hbm": round(dual_bytes / (t_d * 1e-3) / 1e9 / hbm, 4),
                          "algorithmic_bytes": int(dual_bytes)}
     del dY, bufs
+    # output quantized in the GEMM's epilogue against a GEMM then a separate 1x128 pass,
+    # on the dense shape with FP32 scales (the promoted path)
+    wd = workloads.dense()
+    A = _dev_normal((wd.M, wd.K), wd.a_std, 6101)
+    B = _dev_normal((wd.N, wd.K), wd.b_std, 6102)
+    qA, sA = fq.quant_act_1x128(A, False)
+    qB, sB = fq.quant_weight_128x128(B, False)
+    bq = fq.gemm_blockscaled_quant(qA, sA, qB, sB)
+    Cs = torch.empty((wd.M, wd.N), dtype=torch.bfloat16, device="cuda")
+    qs = fq.quant_act_1x128(Cs, False)
+    t_fc = _time_ms(lambda: fq.gemm_blockscaled_quant(qA, sA, qB, sB, out=bq), reps, flush_l2)
+    t_fq = _time_ms(lambda: fq.gemm_blockscaled_quant(qA, sA, qB, sB, out=(None, bq[1], bq[2])),
+                    reps, flush_l2)
+
+    def two_pass():
+        fq.gemm_blockscaled(qA, sA, qB, sB, out=Cs, split_k=False)
+        fq.quant_act_1x128(Cs, False, out=qs)
+
+    t_2 = _time_ms(two_pass, reps, flush_l2)
+    out["gemm_quant_out"] = {"workload": f"dense_{wd.M}x{wd.N}x{wd.K}_fp32_scales_quantized_output",
+                             "fused_with_c_ms": round(t_fc, 4), "fused_codes_only_ms": round(t_fq, 4),
+                             "gemm_then_quant_pass_ms": round(t_2, 4), "launches_fused": 1,
+                             "launches_two_pass": 2}
+    del A, B, qA, sA, qB, sB, bq, Cs, qs
     # FP8 linear layer, one forward + backward (Fprop, Dgrad, Wgrad), dense shapes, pow2
     from fp8_fine_grained_weight_b200.linear import fp8_linear
     Tl, Kl, Nl = 4096, 7168, 7168
@@ -632,7 +656,7 @@ def kernel_rev() -> str:
     ncu counters of a GEMM to the code they measured."""
     import hashlib
     h = hashlib.sha1()
-    for f in ("ptx.cuh", "gemm.cuh", "gemm_ue8m0.cuh", "fp8q.cu"):
+    for f in ("ptx.cuh", "quant.cuh", "gemm.cuh", "gemm_ue8m0.cuh", "fp8q.cu"):
         h.update(open(os.path.join(ROOT, "fp8_fine_grained_weight_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:12]
 

@@ -44,6 +44,9 @@ SIGNATURES = {
                                     _i64, _i64, _i64, _i64, _i64, _i64, _vp]),
     "fp8_gemm_blockscaled_ue8m0": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _i32, _vp, _i32,
                                           _i64, _i64, _i64, _i64, _i64, _i64, _vp]),
+    "fp8_gemm_blockscaled_quant": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _i32, _vp, _i64,
+                                          _vp, _i64, _vp, _i64, _i32, _i64, _i64, _i64, _i64,
+                                          _i64, _vp]),
     "fp8_gemm_grouped_ue8m0": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _i32, _vp, _i32, _i64, _i64,
                                       _i64, _vp]),
     "fp8_gemm_blockscaled_ws": (_i32, [_vp, _vp, _i64, _vp, _vp, _i64, _i32, _vp, _i32,
@@ -297,8 +300,9 @@ def _workspace(device, stream: int, nbytes: int) -> torch.Tensor:
     return ws
 
 
-def _dense_gemm_operands(qa, sa, qb, sb, b_rowwise: bool, out, out_dtype):
-    """Checks of the dense GEMMs' operands; returns (qa, qb, out, M, N, K)."""
+def _dense_gemm_operands(qa, sa, qb, sb, b_rowwise: bool, out, out_dtype, alloc: bool = True):
+    """Checks of the dense GEMMs' operands; returns (qa, qb, out, M, N, K) (out allocated
+    when None and ``alloc``)."""
     qa, qb = _u8(qa), _u8(qb)
     _need(qa, torch.uint8, "qa", 2)
     _need(qb, torch.uint8, "qb", 2)
@@ -314,7 +318,8 @@ def _dense_gemm_operands(qa, sa, qb, sb, b_rowwise: bool, out, out_dtype):
     else:                                                        # [N/128, K/128], pitch implied
         _dense(sb, torch.float32, "sb", (-(-N // 128), K // 128), dev)
     if out is None:
-        out = torch.empty((M, N), dtype=out_dtype, device=dev)
+        if alloc:
+            out = torch.empty((M, N), dtype=out_dtype, device=dev)
     else:
         _out_code(out.dtype)
         _rows(out, out.dtype, "out", M, N, dev)
@@ -347,6 +352,38 @@ def gemm_blockscaled(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: t
               BSCALE_ROW if b_rowwise else BSCALE_BLOCK, out.data_ptr(), _out_code(out.dtype),
               M, N, K, qa.stride(0), qb.stride(0), out.stride(0), ws_ptr, ws_len, _stream(qa))
     return out
+
+
+def gemm_blockscaled_quant(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor,
+                           pow2: bool = False, b_rowwise: bool = False, with_c: bool = True,
+                           out=None):
+    """bf16 C = A B^T with per-128-K promotion, also quantized 1x128 in the GEMM's epilogue.
+
+    Same operands as ``gemm_blockscaled``.  Returns (C bf16 [M, N] or None without
+    ``with_c``, qc uint8 [M, N], sc fp32 [N/128, M]) where (qc, sc) equals
+    ``quant_act_1x128(C, pow2)``.  ``out``: (C or None, qc, sc) to write into.
+    """
+    if out is None:
+        qa, qb, c, M, N, K = _dense_gemm_operands(qa, sa, qb, sb, b_rowwise, None, torch.bfloat16,
+                                                  alloc=with_c)
+        qc = torch.empty((M, N), dtype=torch.uint8, device=qa.device)
+        sc = torch.empty((N // 128, M), dtype=torch.float32, device=qa.device)
+    else:
+        c, qc, sc = out
+        if c is not None and c.dtype != torch.bfloat16:
+            raise ValueError("C must be bf16")
+        qa, qb, c, M, N, K = _dense_gemm_operands(qa, sa, qb, sb, b_rowwise, c, torch.bfloat16,
+                                                  alloc=False)
+        _rows(_u8(qc), torch.uint8, "qc", M, N, qa.device)
+        _rows(sc, torch.float32, "sc", N // 128, M, qa.device)
+    with _on(qa):
+        _call("fp8_gemm_blockscaled_quant", qa.data_ptr(), sa.data_ptr(), sa.stride(0), qb.data_ptr(),
+              sb.data_ptr(), sb.stride(0) if b_rowwise else 0,
+              BSCALE_ROW if b_rowwise else BSCALE_BLOCK, c.data_ptr() if c is not None else None,
+              c.stride(0) if c is not None else 0, _u8(qc).data_ptr(), _u8(qc).stride(0),
+              sc.data_ptr(), sc.stride(0), int(bool(pow2)), M, N, K, qa.stride(0), qb.stride(0),
+              _stream(qa))
+    return c, qc, sc
 
 
 def gemm_blockscaled_ue8m0(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor,

@@ -472,6 +472,34 @@ int fp8_gemm_blockscaled(const uint8_t* A, const float* sA, int64_t ld_sa, const
                                  lda, ldb, ldc, nullptr, 0, stream);
 }
 
+int fp8_gemm_blockscaled_quant(const uint8_t* A, const float* sA, int64_t ld_sa, const uint8_t* B,
+                               const float* sB, int64_t ld_sb, int b_scale_mode, void* C, int64_t ldc,
+                               uint8_t* qC, int64_t ldq, float* sC, int64_t ld_sc, int pow2_scale,
+                               int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
+                               void* stream) {
+  if (M == 0 && N >= 0 && K >= 0) return FP8Q_OK;
+  // C is optional: without it the C checks run on stand-ins that always pass them.
+  int st = check_dense_blockscaled(A, sA, ld_sa, B, sB, ld_sb, b_scale_mode,
+                                   C != nullptr ? C : static_cast<void*>(qC), FP8Q_OUT_BF16, M, N,
+                                   K, lda, ldb, C != nullptr ? ldc : N);
+  if (st != FP8Q_OK) return st;
+  if (!qC || !sC) return FP8Q_ERR_NULL;
+  if (ldq < N || ld_sc < M) return FP8Q_ERR_SHAPE;
+  if (ldq % 16 != 0 || !aligned(qC, 16) || !aligned(sC, 4)) return FP8Q_ERR_ALIGN;
+  CUtensorMap tmA, tmB;
+  if ((st = encode_operand(&tmA, A, K, M, lda, 128)) != FP8Q_OK) return st;
+  if ((st = encode_operand(&tmB, B, K, N, ldb, Cfg1::kBBox)) != FP8Q_OK) return st;
+  GemmArgs a{};
+  a.sA = sA; a.ld_sa = ld_sa; a.sB = sB; a.ld_sb = ld_sb; a.C = C; a.ldc = ldc;
+  a.M = M; a.N = N; a.G = static_cast<int>(K / 128); a.m_offsets = nullptr; a.num_experts = 0;
+  a.qc = qC; a.ldq = ldq; a.sc = sC; a.ld_sc = ld_sc; a.qpow2 = pow2_scale != 0;
+  const int64_t tiles = dense_tiles(M, N);
+  if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
+  // no workspace: every tile is finished by one CTA, which quantizes its rows
+  return dispatch_dense(tmA, tmB, a, b_scale_mode == FP8Q_BSCALE_ROW1x128, true, tiles, nullptr, 0,
+                        static_cast<cudaStream_t>(stream));
+}
+
 int fp8_gemm_blockscaled_ue8m0(const uint8_t* A, const float* sA, int64_t ld_sa,
                                const uint8_t* B, const float* sB, int64_t ld_sb, int b_scale_mode,
                                void* C, int out_dtype, int64_t M, int64_t N, int64_t K,

@@ -52,6 +52,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace fp8q {
 
@@ -93,6 +94,15 @@ struct GemmArgs {
   int tiles_full;
   int tail_tiles;
   int tail_split;
+  // Quantized output (dense, bf16, no split): when qc is set, every 1x128 row segment of
+  // the bf16 C is also quantized as fp8q_quant_act_1x128 would (codes qc[m * ldq + n],
+  // scales sc[(n / 128) * ld_sc + m], power-of-two scales when qpow2); C itself is
+  // stored only when C is set.
+  uint8_t* qc;
+  int64_t ldq;
+  float* sc;
+  int64_t ld_sc;
+  int qpow2;
 };
 
 // A unit of work of one CTA (or CTA pair): a tile and a range of its K-groups, written
@@ -247,6 +257,43 @@ __device__ __forceinline__ void promote_chunk(float2* acc, const uint32_t* r, fl
       a0 = __ffma2_rn(p0, sc2, a0);
       a1 = __ffma2_rn(p1, sc2, a1);
     }
+  }
+}
+
+// Stores a row segment held one row per lane: lane i of each quad (4 lanes, rows r0 .. r0 + 3)
+// holds chunks v[0 .. NC) (16 bytes each) of its row, destined for row_ptr(row) + 16 c.
+// Groups of four chunks are transposed inside the quad (shuffles), so that each store
+// instruction writes 64 contiguous bytes of one row per quad: 8 row pieces per warp
+// instruction instead of 32 scattered 16-byte pieces.  `valid` is whether this lane's row
+// is inside C; the quad's rows are exchanged with it.
+template <int NC>
+__device__ __forceinline__ void store_rows_by_quads(uint4 (&v)[NC], uint8_t* my_row, bool valid) {
+  static_assert(NC % 4 == 0, "groups of four chunks");
+  const int lane = threadIdx.x & 31, i = lane & 3;
+  uint8_t* rows[4];
+  bool ok[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {          // the quad's rows, row k from lane 4 (lane / 4) + k
+    rows[k] = reinterpret_cast<uint8_t*>(
+        __shfl_sync(0xFFFFFFFFu, reinterpret_cast<uintptr_t>(my_row), (lane & ~3) + k));
+    ok[k] = __shfl_sync(0xFFFFFFFFu, valid, (lane & ~3) + k);
+  }
+#pragma unroll
+  for (int c0 = 0; c0 < NC; c0 += 4) {
+    uint32_t w[4][4];                      // w[word][j]: word of chunk c0 + j
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      w[0][j] = v[c0 + j].x;
+      w[1][j] = v[c0 + j].y;
+      w[2][j] = v[c0 + j].z;
+      w[3][j] = v[c0 + j].w;
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x) quad_transpose4(w[x], i);   // now w[x][k]: chunk c0 + i of row k
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (ok[k])
+        *reinterpret_cast<uint4*>(rows[k] + 16 * (c0 + i)) = make_uint4(w[0][k], w[1][k], w[2][k], w[3][k]);
   }
 }
 
@@ -576,28 +623,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int j = 0; j < kSetCols / 2; j += 2)
           *reinterpret_cast<float4*>(wrow + 2 * j) =
               make_float4(acc[j].x, acc[j].y, acc[j + 1].x, acc[j + 1].y);
-      } else if (ok && row_ok && cols_ok) {
+      } else if (ok && cols_ok) {          // warp-uniform: the row stores shuffle inside quads
         if (OUT_BF16) {
-          __nv_bfloat16* crow = reinterpret_cast<__nv_bfloat16*>(p.C) + m * p.ldc + n0;
+          // hv[j]: columns 8j .. 8j + 7 of the row segment, rounded to bf16
+          uint4 hv[kSetCols / 8];
 #pragma unroll
-          for (int j = 0; j < kSetCols / 2; j += 4) {
-            __nv_bfloat162 h0 = __float22bfloat162_rn(acc[j + 0]);
-            __nv_bfloat162 h1 = __float22bfloat162_rn(acc[j + 1]);
-            __nv_bfloat162 h2 = __float22bfloat162_rn(acc[j + 2]);
-            __nv_bfloat162 h3 = __float22bfloat162_rn(acc[j + 3]);
-            uint4 o;
-            o.x = *reinterpret_cast<uint32_t*>(&h0);
-            o.y = *reinterpret_cast<uint32_t*>(&h1);
-            o.z = *reinterpret_cast<uint32_t*>(&h2);
-            o.w = *reinterpret_cast<uint32_t*>(&h3);
-            *reinterpret_cast<uint4*>(crow + 2 * j) = o;
+          for (int j = 0; j < kSetCols / 8; ++j) {
+            __nv_bfloat162 h0 = __float22bfloat162_rn(acc[4 * j + 0]);
+            __nv_bfloat162 h1 = __float22bfloat162_rn(acc[4 * j + 1]);
+            __nv_bfloat162 h2 = __float22bfloat162_rn(acc[4 * j + 2]);
+            __nv_bfloat162 h3 = __float22bfloat162_rn(acc[4 * j + 3]);
+            hv[j].x = *reinterpret_cast<uint32_t*>(&h0);
+            hv[j].y = *reinterpret_cast<uint32_t*>(&h1);
+            hv[j].z = *reinterpret_cast<uint32_t*>(&h2);
+            hv[j].w = *reinterpret_cast<uint32_t*>(&h3);
+          }
+          if (p.C != nullptr)
+            store_rows_by_quads(hv, reinterpret_cast<uint8_t*>(reinterpret_cast<__nv_bfloat16*>(p.C) + m * p.ldc + n0),
+                                row_ok);
+          if (p.qc != nullptr) {
+            // this thread's segment is exactly one 1x128 tile of the output row
+            static_assert(kSetCols == 128, "one 1x128 output tile per epilogue thread");
+            const float s_out = tile_scale(amax_vectors<kSetCols / 8>(hv), p.qpow2 != 0);
+            uint2 o[kSetCols / 8];
+            quant_vectors<kSetCols / 8>(hv, Quotient(s_out), o);
+            uint4 qv[kSetCols / 16];
+#pragma unroll
+            for (int j = 0; j < kSetCols / 16; ++j)
+              qv[j] = make_uint4(o[2 * j].x, o[2 * j].y, o[2 * j + 1].x, o[2 * j + 1].y);
+            store_rows_by_quads(qv, p.qc + m * p.ldq + n0, row_ok);
+            if (row_ok) p.sc[(n0 / 128) * p.ld_sc + m] = s_out;
           }
         } else {
-          float* crow = reinterpret_cast<float*>(p.C) + m * p.ldc + n0;
+          uint4 fv[kSetCols / 4];
 #pragma unroll
-          for (int j = 0; j < kSetCols / 2; j += 2)
-            *reinterpret_cast<float4*>(crow + 2 * j) =
-                make_float4(acc[j].x, acc[j].y, acc[j + 1].x, acc[j + 1].y);
+          for (int j = 0; j < kSetCols / 4; ++j)
+            fv[j] = make_uint4(__float_as_uint(acc[2 * j].x), __float_as_uint(acc[2 * j].y),
+                               __float_as_uint(acc[2 * j + 1].x), __float_as_uint(acc[2 * j + 1].y));
+          store_rows_by_quads(fv, reinterpret_cast<uint8_t*>(reinterpret_cast<float*>(p.C) + m * p.ldc + n0),
+                              row_ok);
         }
       }
     }

@@ -154,6 +154,31 @@ int fp8_gemm_blockscaled(const uint8_t* A, const float* sA, int64_t ld_sa, const
                          void* stream);
 
 /*
+ * fp8_gemm_blockscaled with bf16 output whose result is also quantized in 1x128 tiles
+ * inside the GEMM's epilogue, for a following FP8 GEMM.  why-be.co.kr wr_id=57820 para 4
+ * describes the HBM round trip of a separate quantization pass (read the bf16 values
+ * back, write FP8 and scales) and asks for the FP8 cast to be fused with the memory
+ * access; here it is fused into the producing kernel: each epilogue thread holds one row's
+ * 128-column segment of the output tile, exactly one 1x128 tile.
+ *
+ * Results (bit-exact contract):
+ *   Cb = the bf16 C of fp8_gemm_blockscaled (FP8Q_OUT_BF16) for the same arguments;
+ *   (qC, sC) = fp8q_quant_act_1x128(Cb, pow2_scale): codes qC[m * ldq + n], scales
+ *   sC[(n / 128) * ld_sc + m] (group-major, as the quantizer writes them).
+ * C   device bf16 [M, N], row stride ldc elements, or NULL: then Cb is not stored
+ * qC  device E4M3 [M, N], row stride ldq bytes        sC device fp32 [N/128][ld_sc]
+ * Requires everything fp8_gemm_blockscaled requires (for C only when C is set), qC and sC
+ * non-NULL, ldq >= N and a multiple of 16, qC 16-byte aligned, ld_sc >= M, sC 4-byte
+ * aligned; otherwise an error before any launch.  No workspace: the last partial wave is
+ * not split along K.
+ */
+int fp8_gemm_blockscaled_quant(const uint8_t* A, const float* sA, int64_t ld_sa, const uint8_t* B,
+                               const float* sB, int64_t ld_sb, int b_scale_mode, void* C, int64_t ldc,
+                               uint8_t* qC, int64_t ldq, float* sC, int64_t ld_sc, int pow2_scale,
+                               int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
+                               void* stream);
+
+/*
  * fp8_gemm_blockscaled for power-of-two scales, with the scaling done inside the tensor
  * core.  why-be.co.kr wr_id=57820 para 4 and why-be.co.kr wr_id=72410 para 3 ask for
  * tensor cores that receive the scaling factors and run the MMA with group scaling; on

@@ -171,6 +171,33 @@ def test_gemm_validation(L, entry):
     assert call(ldc=260, out=0) == 3           # 520 B row pitch is not a multiple of 16
 
 
+def test_gemm_quant_validation(L):
+    f = L.fp8_gemm_blockscaled_quant
+    ok_args = dict(A=P16, sA=P16, ld_sa=256, B=P16, sB=P16, ld_sb=0, mode=0, C=P16, ldc=256,
+                   qC=P16, ldq=256, sC=P16, ld_sc=256, pow2=0, M=256, N=256, K=256, lda=256,
+                   ldb=256)
+
+    def call(**kw):
+        a = dict(ok_args, **kw)
+        return f(a["A"], a["sA"], a["ld_sa"], a["B"], a["sB"], a["ld_sb"], a["mode"], a["C"],
+                 a["ldc"], a["qC"], a["ldq"], a["sC"], a["ld_sc"], a["pow2"], a["M"], a["N"],
+                 a["K"], a["lda"], a["ldb"], NULL)
+
+    assert call(M=0) == 0                      # empty problem: no-op
+    assert call(A=NULL) == 1
+    assert call(qC=NULL) == 1
+    assert call(sC=NULL) == 1
+    assert call(C=NULL, qC=NULL) == 1          # the codes are not optional
+    assert call(N=200) == 2                    # N % 128
+    assert call(ldq=128) == 2                  # ldq < N
+    assert call(ld_sc=100) == 2                # ld_sc < M
+    assert call(ldc=128) == 2                  # ldc < N (C given)
+    assert call(ldq=264) == 3                  # not a multiple of 16
+    assert call(qC=P_MIS) == 3
+    assert call(ldc=260) == 3                  # 520 B row pitch is not a multiple of 16
+    assert call(mode=7) == 4
+
+
 @pytest.mark.parametrize("entry", ["fp8_gemm_grouped", "fp8_gemm_grouped_ue8m0"])
 def test_grouped_validation(L, entry):
     f = getattr(L, entry)

@@ -163,6 +163,25 @@ def test_gemm_ue8m0_and_nopromo_guard(fq, rowwise, M):
         Cn.check("gemm_nopromo")
 
 
+@pytest.mark.parametrize("with_c", [True, False])
+def test_gemm_quant_out_guard(fq, with_c):
+    """The GEMM that also quantizes its output: C (optional), the codes (pitch > N) and the
+    group-major scales (pitch > M); N = 384 leaves the last tile's second half outside."""
+    import torch
+    M, N, K = 300, 384, 512
+    qa, sa, qb, sb = _gemm_operands(fq, M, N, K, 41)
+    C = Guarded(M, N, N + 64, torch.bfloat16) if with_c else None
+    q = Guarded(M, N, N + 48, torch.uint8)
+    s = Guarded(N // 128, M, M + 20, torch.float32)
+    fq.gemm_blockscaled_quant(qa, sa, qb, sb, out=(C.view if with_c else None, q.view, s.view))
+    torch.cuda.synchronize()
+    assert fq.device_error() == 0
+    if with_c:
+        C.check("gemm_blockscaled_quant C")
+    q.check("gemm_blockscaled_quant codes")
+    s.check("gemm_blockscaled_quant scales")
+
+
 def test_noalloc_guard(fq):
     import torch
     M, N, K = 300, 1024, 2048          # splits its last wave: the fixed scratch is used
