@@ -407,30 +407,55 @@ __global__ void __launch_bounds__(Ue8m0Cfg<GROUPED>::kThreads, 1)
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + buf * kN +
                              set * Cfg::kSetCols;
       const int64_t n_set = tl.col0 + set * Cfg::kSetCols;
+      const bool row_ok = m < tl.row_end;
+      uint8_t* crow = reinterpret_cast<uint8_t*>(p.C) + (m * p.ldc + n_set) * (OUT_BF16 ? 2 : 4);
+      // Stores go through store_rows_by_quads (64 contiguous bytes of 8 rows per warp
+      // instruction): bf16 in 32-column steps, fp32 in 16-column steps; a bf16 step that
+      // would cross N, and the set's last 16 bf16 columns, store 32 bytes per row directly.
+      // Every condition on columns is warp-uniform (n_set is the warp's).
 #pragma unroll 1
-      for (int c = 0; c < Cfg::kSetCols; c += 16) {
+      for (int c = 0; c < Cfg::kSetCols; c += (OUT_BF16 && c + 32 <= Cfg::kSetCols) ? 32 : 16) {
+        const int64_t n0 = n_set + c;
+        if (OUT_BF16 && c + 32 <= Cfg::kSetCols && n0 + 32 <= p.N) {
+          uint32_t r[32];
+          tmem_ld_32cols(taddr + c, r);
+          tmem_ld_wait();
+          uint4 hv[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint32_t h[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(r[8 * j + 2 * t]),
+                                                       __uint_as_float(r[8 * j + 2 * t + 1]));
+              h[t] = *reinterpret_cast<uint32_t*>(&v);
+            }
+            hv[j] = make_uint4(h[0], h[1], h[2], h[3]);
+          }
+          store_rows_by_quads(hv, crow + 2 * c, row_ok);
+          continue;
+        }
         uint32_t r[16];
         tmem_ld_16cols(taddr + c, r);
         tmem_ld_wait();
-        const int64_t n0 = n_set + c;
-        if (m < tl.row_end && n0 < p.N) {                // N % 16 == 0: whole chunks
-          if (OUT_BF16) {
+        if (n0 >= p.N) continue;                         // N % 16 == 0: whole 16-column chunks
+        if (OUT_BF16) {
+          if (row_ok) {
             uint32_t h[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
               __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
               h[j] = *reinterpret_cast<uint32_t*>(&v);
             }
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.C) + m * p.ldc + n0);
+            uint4* dst = reinterpret_cast<uint4*>(crow + 2 * c);
             dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
             dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
-          } else {
-            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.C) + m * p.ldc + n0);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                   __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
           }
+        } else {
+          uint4 fv[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) fv[j] = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+          store_rows_by_quads(fv, crow + 4 * c, row_ok);
         }
       }
       tc_fence_before();
