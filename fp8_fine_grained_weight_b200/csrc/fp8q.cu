@@ -67,10 +67,10 @@ int encode_operand(CUtensorMap* tm, const void* base, uint64_t K, uint64_t rows,
 // B scale modes).
 using Cfg1 = fp8q::GemmCfg<false>;
 
-template <bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16>
+template <bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16, bool QOUT = false>
 struct GemmLauncher {
   using Cfg = fp8q::GemmCfg<ROW_B>;
-  static constexpr auto kern = fp8q::gemm_fp8_blockscaled_kernel<PROMOTE, ROW_B, GROUPED, OUT_BF16>;
+  static constexpr auto kern = fp8q::gemm_fp8_blockscaled_kernel<PROMOTE, ROW_B, GROUPED, OUT_BF16, QOUT>;
 
   // Co-resident CTAs on the current device; sets the kernel's attributes on first use.
   // 0 on failure.
@@ -162,10 +162,10 @@ int check_dense_blockscaled(const uint8_t* A, const float* sA, int64_t ld_sa, co
 // Launch one GEMM instantiation.  work: tiles (a bound for grouped).  Dense GEMMs given a
 // large enough workspace split their last partial wave along K and finish with a
 // reduction launch on the same stream.
-template <bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16>
+template <bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16, bool QOUT = false>
 int run_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, GemmArgs a, int64_t work,
              void* ws, size_t ws_bytes, cudaStream_t st) {
-  using L = GemmLauncher<PROMOTE, ROW_B, GROUPED, OUT_BF16>;
+  using L = GemmLauncher<PROMOTE, ROW_B, GROUPED, OUT_BF16, QOUT>;
   const int units = L::max_units();
   if (units <= 0) return FP8Q_ERR_CUDA;
   a.ws = nullptr;
@@ -191,9 +191,14 @@ int run_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, GemmArgs a, int64_t
   return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
-// Promoted dense GEMM: B scale mode and output type chosen at run time.
+// Promoted dense GEMM: B scale mode and output type chosen at run time; a quantized
+// output (bf16, no workspace) takes its own instantiation.
 int dispatch_dense(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, bool row_b,
                    bool bf16, int64_t work, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (a.qc != nullptr) {
+    return row_b ? run_gemm<true, true, false, true, true>(tmA, tmB, a, work, nullptr, 0, st)
+                 : run_gemm<true, false, false, true, true>(tmA, tmB, a, work, nullptr, 0, st);
+  }
   if (row_b) {
     return bf16 ? run_gemm<true, true, false, true>(tmA, tmB, a, work, ws, ws_bytes, st)
                 : run_gemm<true, true, false, false>(tmA, tmB, a, work, ws, ws_bytes, st);
@@ -457,6 +462,7 @@ int fp8_gemm_blockscaled_ws(const uint8_t* A, const float* sA, int64_t ld_sa, co
   GemmArgs a{};
   a.sA = sA; a.ld_sa = ld_sa; a.sB = sB; a.ld_sb = ld_sb; a.C = C; a.ldc = ldc;
   a.M = M; a.N = N; a.G = static_cast<int>(K / 128); a.m_offsets = nullptr; a.num_experts = 0;
+  a.n_fastest = M > N;
   const int64_t tiles = dense_tiles(M, N);
   if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   const bool row_b = b_scale_mode == FP8Q_BSCALE_ROW1x128, bf16 = out_dtype == FP8Q_OUT_BF16;
@@ -492,6 +498,7 @@ int fp8_gemm_blockscaled_quant(const uint8_t* A, const float* sA, int64_t ld_sa,
   GemmArgs a{};
   a.sA = sA; a.ld_sa = ld_sa; a.sB = sB; a.ld_sb = ld_sb; a.C = C; a.ldc = ldc;
   a.M = M; a.N = N; a.G = static_cast<int>(K / 128); a.m_offsets = nullptr; a.num_experts = 0;
+  a.n_fastest = M > N;
   a.qc = qC; a.ldq = ldq; a.sc = sC; a.ld_sc = ld_sc; a.qpow2 = pow2_scale != 0;
   const int64_t tiles = dense_tiles(M, N);
   if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
@@ -515,6 +522,7 @@ int fp8_gemm_blockscaled_ue8m0(const uint8_t* A, const float* sA, int64_t ld_sa,
   GemmArgs a{};
   a.sA = sA; a.ld_sa = ld_sa; a.sB = sB; a.ld_sb = ld_sb; a.C = C; a.ldc = ldc;
   a.M = M; a.N = N; a.G = static_cast<int>(K / 128); a.m_offsets = nullptr; a.num_experts = 0;
+  a.n_fastest = M > N;
   const int64_t tiles = ((M + Cfg::kTileM - 1) / Cfg::kTileM) * ((N + Cfg::kN - 1) / Cfg::kN);
   if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   const auto s = static_cast<cudaStream_t>(stream);
@@ -613,6 +621,7 @@ int fp8_gemm_nopromo(const uint8_t* A, const float* sA, const uint8_t* B, const 
   GemmArgs a{};
   a.sA = sA; a.ld_sa = 0; a.sB = sB; a.ld_sb = 0; a.C = C; a.ldc = ldc;
   a.M = M; a.N = N; a.G = static_cast<int>(K / 128); a.m_offsets = nullptr; a.num_experts = 0;
+  a.n_fastest = M > N;
   const int64_t tiles = dense_tiles(M, N);
   if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   return run_gemm<false, false, false, false>(tmA, tmB, a, tiles, nullptr, 0,

@@ -103,6 +103,10 @@ struct GemmArgs {
   float* sc;
   int64_t ld_sc;
   int qpow2;
+  // Dense tile order: m fastest (0), so that the CTAs of a wave share B tiles and re-read
+  // A once per wave, or n fastest (1), the reverse; the host takes n fastest when A is
+  // the larger operand (M > N).
+  int n_fastest;
 };
 
 // A unit of work of one CTA (or CTA pair): a tile and a range of its K-groups, written
@@ -203,7 +207,9 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmArgs& p, int mt_tot
                                             const int* sched) {
   Tile tl;
   if (!GROUPED) {
-    const int mt = t % mt_total, nt = t / mt_total;
+    const int fast = p.n_fastest ? nt_total : mt_total;   // tiles along the fast axis
+    const int q = t / fast, r = t - q * fast;
+    const int mt = p.n_fastest ? q : r, nt = p.n_fastest ? r : q;
     tl.row0 = static_cast<int64_t>(mt) * TILE_M;
     tl.row_end = p.M;
     tl.col0 = static_cast<int64_t>(nt) * TILE_N;
@@ -297,7 +303,10 @@ __device__ __forceinline__ void store_rows_by_quads(uint4 (&v)[NC], uint8_t* my_
   }
 }
 
-template <bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16>
+// QOUT: the bf16 output is also quantized in 1x128 tiles (codes and scales through
+// p.qc / p.sc; C only when p.C is set); a separate instantiation, so that the plain
+// GEMM's registers are not shaped by it.
+template <bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16, bool QOUT = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_fp8_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA,
                                 const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
@@ -641,12 +650,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (p.C != nullptr)
             store_rows_by_quads(hv, reinterpret_cast<uint8_t*>(reinterpret_cast<__nv_bfloat16*>(p.C) + m * p.ldc + n0),
                                 row_ok);
-          if (p.qc != nullptr) {
+          if constexpr (QOUT) {
             // this thread's segment is exactly one 1x128 tile of the output row
-            static_assert(kSetCols == 128, "one 1x128 output tile per epilogue thread");
+            static_assert(kSetCols == 128 && !GROUPED, "one 1x128 output tile per epilogue thread");
             const float s_out = tile_scale(amax_vectors<kSetCols / 8>(hv), p.qpow2 != 0);
             uint2 o[kSetCols / 8];
-            quant_vectors<kSetCols / 8>(hv, Quotient(s_out), o);
+            // f32x2 quotients, the rule voted once per warp (every lane's row has its own
+            // tile scale)
+            with_pair_quotient<true>(Quotient(s_out), [&](const auto& qd) {
+#pragma unroll
+              for (int j = 0; j < kSetCols / 8; ++j) {
+                const float2 p0 = qd(hv[j].x), p1 = qd(hv[j].y), p2 = qd(hv[j].z), p3 = qd(hv[j].w);
+                o[j].x = __byte_perm(cvt_e4m3x2(p0.x, p0.y), cvt_e4m3x2(p1.x, p1.y), 0x5410);
+                o[j].y = __byte_perm(cvt_e4m3x2(p2.x, p2.y), cvt_e4m3x2(p3.x, p3.y), 0x5410);
+              }
+            });
             uint4 qv[kSetCols / 16];
 #pragma unroll
             for (int j = 0; j < kSetCols / 16; ++j)
@@ -683,8 +701,9 @@ template <bool OUT_BF16, int TILE_M, int TILE_N>
 __global__ void __launch_bounds__(TILE_N) splitk_reduce_kernel(const GemmArgs p, int mt_total) {
   const int r = blockIdx.x / TILE_M, row = blockIdx.x % TILE_M, col = threadIdx.x;
   const int t = p.tiles_full + r;
-  const int64_t m = static_cast<int64_t>(t % mt_total) * TILE_M + row;
-  const int64_t n = static_cast<int64_t>(t / mt_total) * TILE_N + col;
+  const int nt_total = static_cast<int>((p.N + TILE_N - 1) / TILE_N);
+  const int64_t m = static_cast<int64_t>(p.n_fastest ? t / nt_total : t % mt_total) * TILE_M + row;
+  const int64_t n = static_cast<int64_t>(p.n_fastest ? t % nt_total : t / mt_total) * TILE_N + col;
   const float* w = p.ws + (static_cast<int64_t>(r) * p.tail_split * TILE_M + row) * TILE_N + col;
   float acc = 0.0f;
   for (int c = 0; c < p.tail_split; ++c) acc += w[static_cast<int64_t>(c) * TILE_M * TILE_N];

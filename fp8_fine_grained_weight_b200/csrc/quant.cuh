@@ -264,36 +264,51 @@ __device__ __forceinline__ uint32_t dual_chunk(uint32_t tile, uint32_t r, uint32
 // x / s for two values, one rule of Quotient each, f32x2 where the rule allows.  A pass
 // picks the rule once per warp (every lane's tile agrees on it: a vote), so the loops
 // carry no per-element branches; the general form remains for warps whose tiles differ.
-// Pair quotients take the NEGATED pair nx = (-x0, -x1) (bf16lo_neg / bf16hi_neg) and
-// return (x0 / s, x1 / s) rounded as Quotient does; the f32x2 instructions then need no
-// operand negation.
+// Pair quotients: (lo / s, hi / s) of the two bf16 values of a 32-bit word, rounded as
+// Quotient does.  NEG: the word is unpacked to the negated values (-x), which the
+// corrected rule's f32x2 instructions take without operand negation; the FP32-scale
+// kernels use it (measured faster there), the power-of-two ones unpack x itself.
+template <bool NEG>
+__device__ __forceinline__ float2 unpack_pair(uint32_t w) {
+  if constexpr (NEG) return make_float2(bf16lo_neg(w), bf16hi_neg(w));
+  else return make_float2(bf16lo(w), bf16hi(w));
+}
+template <bool NEG>
 struct PairExact {              // s a power of two: x * (1/s) exactly
-  float2 nr2;
-  __device__ __forceinline__ explicit PairExact(const Quotient& q) : nr2(make_float2(-q.r, -q.r)) {}
-  __device__ __forceinline__ float2 operator()(float2 nx) const { return __fmul2_rn(nx, nr2); }
+  float2 r2;
+  __device__ __forceinline__ explicit PairExact(const Quotient& q)
+      : r2(make_float2(NEG ? -q.r : q.r, NEG ? -q.r : q.r)) {}
+  __device__ __forceinline__ float2 operator()(uint32_t w) const { return __fmul2_rn(unpack_pair<NEG>(w), r2); }
 };
+template <bool NEG>
 struct PairCorrected {          // Markstein's correction with the rounded reciprocal
   float2 nr2, s2;
   __device__ __forceinline__ explicit PairCorrected(const Quotient& q)
       : nr2(make_float2(-q.r, -q.r)), s2(make_float2(q.s, q.s)) {}
-  __device__ __forceinline__ float2 operator()(float2 nx) const {
+  __device__ __forceinline__ float2 operator()(uint32_t w) const {
+    float2 nx = unpack_pair<NEG>(w);
+    if constexpr (!NEG) nx = make_float2(-nx.x, -nx.y);
     const float2 q0 = __fmul2_rn(nx, nr2);      // RN(x r)
     const float2 d = __ffma2_rn(q0, s2, nx);    // q0 s - x, exact
     return __ffma2_rn(d, nr2, q0);              // RN(q0 - d r)
   }
 };
+template <bool NEG>
 struct PairGeneral {            // any rule, decided per call
   Quotient q;
   __device__ __forceinline__ explicit PairGeneral(const Quotient& q_) : q(q_) {}
-  __device__ __forceinline__ float2 operator()(float2 nx) const { return make_float2(q(-nx.x), q(-nx.y)); }
+  __device__ __forceinline__ float2 operator()(uint32_t w) const {
+    const float2 x = unpack_pair<NEG>(w);
+    return NEG ? make_float2(q(-x.x), q(-x.y)) : make_float2(q(x.x), q(x.y));
+  }
 };
 
 // Runs body(pair quotient of the calling lane's tile) with the rule picked once per warp.
-template <typename Body>
+template <bool NEG, typename Body>
 __device__ __forceinline__ void with_pair_quotient(const Quotient& q, Body body) {
-  if (__all_sync(0xffffffffu, q.mode == kCorrected)) body(PairCorrected(q));
-  else if (__all_sync(0xffffffffu, q.mode == kExactRcp)) body(PairExact(q));
-  else body(PairGeneral(q));
+  if (__all_sync(0xffffffffu, q.mode == kCorrected)) body(PairCorrected<NEG>(q));
+  else if (__all_sync(0xffffffffu, q.mode == kExactRcp)) body(PairExact<NEG>(q));
+  else body(PairGeneral<NEG>(q));
 }
 
 // In-quad 4x4 transpose of 32-bit words: lane q of a group of 4 lanes holds row q of a
@@ -371,14 +386,14 @@ __global__ void __launch_bounds__(256, 6) quant_act_dual_kernel(const __grid_con
     a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
     const float sc = tile_scale(a, POW2);
     uint8_t* dst = q + m * ldq + k0;
-    with_pair_quotient(Quotient(sc), [&](const auto& qd) {
+    with_pair_quotient<!POW2>(Quotient(sc), [&](const auto& qd) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const uint4 w = v[j];
-        const float2 p0 = qd(make_float2(bf16lo_neg(w.x), bf16hi_neg(w.x)));
-        const float2 p1 = qd(make_float2(bf16lo_neg(w.y), bf16hi_neg(w.y)));
-        const float2 p2 = qd(make_float2(bf16lo_neg(w.z), bf16hi_neg(w.z)));
-        const float2 p3 = qd(make_float2(bf16lo_neg(w.w), bf16hi_neg(w.w)));
+        const float2 p0 = qd(w.x);
+        const float2 p1 = qd(w.y);
+        const float2 p2 = qd(w.z);
+        const float2 p3 = qd(w.w);
         uint2 o;
         o.x = __byte_perm(cvt_e4m3x2(p0.x, p0.y), cvt_e4m3x2(p1.x, p1.y), 0x5410);
         o.y = __byte_perm(cvt_e4m3x2(p2.x, p2.y), cvt_e4m3x2(p3.x, p3.y), 0x5410);
@@ -409,11 +424,11 @@ __global__ void __launch_bounds__(256, 6) quant_act_dual_kernel(const __grid_con
     const float sc = tile_scale(a, POW2);
     // pairs of codes: rows 8b + 2 l4 (low byte) and 8b + 2 l4 + 1
     uint32_t vv[8];                            // vv[c]: rows 16c + 2 l4, +1 | 16c + 8 + 2 l4, +1
-    with_pair_quotient(Quotient(sc), [&](const auto& qd) {
+    with_pair_quotient<!POW2>(Quotient(sc), [&](const auto& qd) {
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        const float2 e0 = qd(make_float2(bf16lo_neg(w2[2 * c]), bf16hi_neg(w2[2 * c])));
-        const float2 e1 = qd(make_float2(bf16lo_neg(w2[2 * c + 1]), bf16hi_neg(w2[2 * c + 1])));
+        const float2 e0 = qd(w2[2 * c]);
+        const float2 e1 = qd(w2[2 * c + 1]);
         vv[c] = __byte_perm(cvt_e4m3x2(e0.x, e0.y), cvt_e4m3x2(e1.x, e1.y), 0x5410);
       }
     });

@@ -6,7 +6,7 @@
  * reciprocal; s >= 2^-92 uses a correctly rounded reciprocal plus one FMA residual
  * correction, with the residual taken as d = q0 s - x and the quotient as RN(q0 - d r)
  * so that x = -0 keeps its sign without a sign restore (the f32x2 path feeds the
- * negated input -x and -r, the same values); smaller s divide.  This program replays
+ * negated input -x and -r, which gives the same values); smaller s divide.  This program replays
  * that sequence with IEEE
  * single-precision host arithmetic (the GPU's fmul/fma/rcp.rn are IEEE too) for
  * every positive finite bf16 amax, both scale modes, and every bf16 x with
@@ -84,9 +84,9 @@ int main(void) {
                     float x = f_of(((uint32_t)xb << 16) | (sg ? 0x80000000u : 0));
                     float ref = x / s;
                     float q;
-                    const float nx = -x, nr = -r;   /* the f32x2 path's operands */
+                    const float nx = -x, nr = -r;   /* the corrected f32x2 path feeds -x, -r */
                     if (mode == 0) {
-                        q = nx * nr;
+                        q = x * r;
                     } else {
                         float q0 = nx * nr;
                         float d = fmaf(q0, s, nx);
