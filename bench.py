@@ -207,6 +207,7 @@ def run_gpu(args, rank, world):
     with ClockSampler(torch.cuda.current_device()) as clk:
         for i in range(args.steps):
             flush_l2()             # outside the step's events
+            torch.cuda._sleep(200_000)   # the host enqueues the step before the GPU reaches it
             step(evs[i])
         torch.cuda.synchronize()
     barrier(world)
@@ -333,22 +334,26 @@ def _spread(ts) -> dict:
 
 def _time_ms(fn, reps, flush_l2, warmup=2):
     """Mean device time of fn() over reps, L2 flushed before each (outside the events).
-    Untimed warm-up calls first: a kernel variant's first launch pays one-time setup."""
+    Untimed warm-up calls first: a kernel variant's first launch pays one-time setup.
+    All reps are enqueued before the host waits, and after each flush the GPU spins for
+    ~0.1 ms, so the host stays ahead of the GPU: host-side latency (a busy host, Python
+    argument checks) never shows up as idle time between a rep's events."""
     import torch
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
-    tot = 0.0
+    evs = []
     for _ in range(reps):
         flush_l2()
+        torch.cuda._sleep(200_000)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         fn()
         e1.record(stream)
-        e1.synchronize()
-        tot += e0.elapsed_time(e1)
-    return tot / reps
+        evs.append((e0, e1))
+    torch.cuda.synchronize()
+    return sum(e0.elapsed_time(e1) for e0, e1 in evs) / reps
 
 
 def _dev_normal(shape, std, seed, outlier_frac=0.0):
@@ -617,6 +622,7 @@ def profile_case(args, name: str, launches: int = 3):
         W = _dev_normal((w.experts, w.N, w.K), w.b_std, 7002)
         qA, sA = fq.quant_act_1x128(A, w.pow2_a or pow2_grouped)
         qW, sW = fq.quant_weight_128x128(W, w.pow2_b or pow2_grouped)
+        del A, W               # keep the captured program's device memory small
         C = torch.empty((w.M, w.N), dtype=torch.bfloat16, device="cuda")
         gemm = fq.gemm_grouped_ue8m0 if pow2_grouped else fq.gemm_grouped
         run = lambda: gemm(qA, sA, qW, sW, off, out=C)
@@ -625,6 +631,7 @@ def profile_case(args, name: str, launches: int = 3):
         B = _dev_normal((w.N, w.K), w.b_std, 7002)
         qA, sA = fq.quant_act_1x128(A, w.pow2_a)
         qB, sB = fq.quant_act_1x128(B, w.pow2_b) if w.b_rowwise else fq.quant_weight_128x128(B, w.pow2_b)
+        del A, B
         C = torch.empty((w.M, w.N), dtype=torch.float32 if w.out_fp32 else torch.bfloat16, device="cuda")
         if gemm_path(args, w) == "ue8m0":
             run = lambda: fq.gemm_blockscaled_ue8m0(qA, sA, qB, sB, b_rowwise=w.b_rowwise, out=C)
