@@ -315,6 +315,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   constexpr int NB = Cfg::kAccBufs;
   constexpr int kN = Cfg::kN;
   constexpr int kSetCols = Cfg::kSetCols;
+  static_assert(S >= NB, "a stage barrier's phase outlives the epilogue's wait for it");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -452,10 +453,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               mma_f8<1>(d, smem_desc_k_sw128(a_addr + 32 * kk), smem_desc_k_sw128(b_addr + 32 * kk),
                         idesc, accumulate);
             }
-            mma_commit<1>(empty_bar(s));
-            if (publish) {
-              mma_commit<1>(tfull_bar(buf));
+            if (PROMOTE) {
+              // One commit per group: its arrival on the stage's barrier both frees the
+              // stage for the producer and publishes the group's partial to the epilogue
+              // (group it uses stage it % S and accumulator it % NB).
+              mma_commit<1>(empty_bar(s));
               ++acc_it;
+            } else {
+              mma_commit<1>(empty_bar(s));
+              if (publish) {
+                mma_commit<1>(tfull_bar(buf));
+                ++acc_it;
+              }
             }
           }
         }
@@ -559,7 +568,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const float sb_cur = ROW_B ? 0.0f : sring[slot + 128 + set * kSetCols / 128];
           const int sb = slot + 128 + set * kSetCols;        // ROW mode column scales
           const uint32_t buf = acc_it % NB;
-          if (ok) ok = mbar_wait(tfull_bar(buf), (acc_it / NB) & 1u, kSiteEpilogue, abort_flag);
+          // group acc_it's MMAs have completed: the commit on its operand stage's barrier
+          // (the epilogue cannot lag by a phase: group acc_it + S needs the accumulator
+          // that this thread frees after group acc_it + S - NB)
+          if (ok)
+            ok = mbar_wait(empty_bar(acc_it % S), (acc_it / S) & 1u, kSiteEpilogue, abort_flag);
           ok = __all_sync(0xFFFFFFFFu, ok);  // warp-uniform: TMEM loads are per warp
           if (ok && !warp_idle) {
             tc_fence_after();
