@@ -63,14 +63,30 @@ int encode_operand(CUtensorMap* tm, const void* base, uint64_t K, uint64_t rows,
   return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
+// bf16 output C [rows, N] with a row stride of `ldc` elements, stored by TMA: boxes of 64
+// columns (128 bytes) by 32 rows, 128-byte swizzle (the promoted GEMM's staging layout).
+int encode_output_bf16(CUtensorMap* tm, void* base, uint64_t N, uint64_t rows, uint64_t ldc) {
+  auto enc = tensor_map_encoder();
+  if (!enc || !bind_current_context()) return FP8Q_ERR_CUDA;
+  cuuint64_t dims[2] = {N, rows};
+  cuuint64_t strides[1] = {ldc * 2};
+  cuuint32_t box[2] = {64, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
 // Tile shape of the promoted GEMMs: one CTA per 128 x 256 tile (the same shape for both
-// B scale modes).
+// B scale modes and output paths).
 using Cfg1 = fp8q::GemmCfg<false>;
 
 template <bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16, bool QOUT = false>
 struct GemmLauncher {
-  using Cfg = fp8q::GemmCfg<ROW_B>;
+  using Cfg = fp8q::GemmCfgOf<PROMOTE, ROW_B, OUT_BF16, QOUT>;
   static constexpr auto kern = fp8q::gemm_fp8_blockscaled_kernel<PROMOTE, ROW_B, GROUPED, OUT_BF16, QOUT>;
+  static_assert(Cfg::kTileM == Cfg1::kTileM && Cfg::kN == Cfg1::kN, "one tile shape");
 
   // Co-resident CTAs on the current device; sets the kernel's attributes on first use.
   // 0 on failure.
@@ -96,10 +112,10 @@ struct GemmLauncher {
     return units;
   }
 
-  static int launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& args,
-                    int64_t grid, cudaStream_t stream) {
+  static int launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmC,
+                    const GemmArgs& args, int64_t grid, cudaStream_t stream) {
     if (grid <= 0) return FP8Q_OK;
-    kern<<<static_cast<unsigned>(grid), fp8q::kGemmThreads, Cfg::smem_bytes, stream>>>(tmA, tmB, args);
+    kern<<<static_cast<unsigned>(grid), fp8q::kGemmThreads, Cfg::smem_bytes, stream>>>(tmA, tmB, tmC, args);
     return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
   }
 };
@@ -161,10 +177,11 @@ int check_dense_blockscaled(const uint8_t* A, const float* sA, int64_t ld_sa, co
 
 // Launch one GEMM instantiation.  work: tiles (a bound for grouped).  Dense GEMMs given a
 // large enough workspace split their last partial wave along K and finish with a
-// reduction launch on the same stream.
+// reduction launch on the same stream.  tmC: the bf16 output's tensor map for the
+// instantiations that store through TMA (GemmCfgOf's TSTORE), otherwise unused.
 template <bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16, bool QOUT = false>
-int run_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, GemmArgs a, int64_t work,
-             void* ws, size_t ws_bytes, cudaStream_t st) {
+int run_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmC, GemmArgs a,
+             int64_t work, void* ws, size_t ws_bytes, cudaStream_t st) {
   using L = GemmLauncher<PROMOTE, ROW_B, GROUPED, OUT_BF16, QOUT>;
   const int units = L::max_units();
   if (units <= 0) return FP8Q_ERR_CUDA;
@@ -183,7 +200,7 @@ int run_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, GemmArgs a, int64_t
       grid = sp.grid_units;
     }
   }
-  int st_code = L::launch(tmA, tmB, a, grid, st);
+  int st_code = L::launch(tmA, tmB, tmC, a, grid, st);
   if (st_code != FP8Q_OK || a.tail_tiles == 0) return st_code;
   const int mt_total = static_cast<int>((a.M + Cfg1::kTileM - 1) / Cfg1::kTileM);
   fp8q::splitk_reduce_kernel<OUT_BF16, Cfg1::kTileM, Cfg1::kN>
@@ -193,18 +210,19 @@ int run_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, GemmArgs a, int64_t
 
 // Promoted dense GEMM: B scale mode and output type chosen at run time; a quantized
 // output (bf16, no workspace) takes its own instantiation.
-int dispatch_dense(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, bool row_b,
-                   bool bf16, int64_t work, void* ws, size_t ws_bytes, cudaStream_t st) {
+int dispatch_dense(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmC,
+                   const GemmArgs& a, bool row_b, bool bf16, int64_t work, void* ws, size_t ws_bytes,
+                   cudaStream_t st) {
   if (a.qc != nullptr) {
-    return row_b ? run_gemm<true, true, false, true, true>(tmA, tmB, a, work, nullptr, 0, st)
-                 : run_gemm<true, false, false, true, true>(tmA, tmB, a, work, nullptr, 0, st);
+    return row_b ? run_gemm<true, true, false, true, true>(tmA, tmB, tmC, a, work, nullptr, 0, st)
+                 : run_gemm<true, false, false, true, true>(tmA, tmB, tmC, a, work, nullptr, 0, st);
   }
   if (row_b) {
-    return bf16 ? run_gemm<true, true, false, true>(tmA, tmB, a, work, ws, ws_bytes, st)
-                : run_gemm<true, true, false, false>(tmA, tmB, a, work, ws, ws_bytes, st);
+    return bf16 ? run_gemm<true, true, false, true>(tmA, tmB, tmC, a, work, ws, ws_bytes, st)
+                : run_gemm<true, true, false, false>(tmA, tmB, tmC, a, work, ws, ws_bytes, st);
   }
-  return bf16 ? run_gemm<true, false, false, true>(tmA, tmB, a, work, ws, ws_bytes, st)
-              : run_gemm<true, false, false, false>(tmA, tmB, a, work, ws, ws_bytes, st);
+  return bf16 ? run_gemm<true, false, false, true>(tmA, tmB, tmC, a, work, ws, ws_bytes, st)
+              : run_gemm<true, false, false, false>(tmA, tmB, tmC, a, work, ws, ws_bytes, st);
 }
 
 int64_t dense_tiles(int64_t M, int64_t N) {
@@ -466,8 +484,10 @@ int fp8_gemm_blockscaled_ws(const uint8_t* A, const float* sA, int64_t ld_sa, co
   const int64_t tiles = dense_tiles(M, N);
   if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   const bool row_b = b_scale_mode == FP8Q_BSCALE_ROW1x128, bf16 = out_dtype == FP8Q_OUT_BF16;
-  return dispatch_dense(tmA, tmB, a, row_b, bf16, tiles, workspace, workspace_bytes,
-                               static_cast<cudaStream_t>(stream));
+  CUtensorMap tmC = tmA;   // a placeholder unless the output leaves through TMA
+  if (bf16 && !row_b && (st = encode_output_bf16(&tmC, C, N, M, ldc)) != FP8Q_OK) return st;
+  return dispatch_dense(tmA, tmB, tmC, a, row_b, bf16, tiles, workspace, workspace_bytes,
+                        static_cast<cudaStream_t>(stream));
 }
 
 int fp8_gemm_blockscaled(const uint8_t* A, const float* sA, int64_t ld_sa, const uint8_t* B,
@@ -503,7 +523,7 @@ int fp8_gemm_blockscaled_quant(const uint8_t* A, const float* sA, int64_t ld_sa,
   const int64_t tiles = dense_tiles(M, N);
   if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   // no workspace: every tile is finished by one CTA, which quantizes its rows
-  return dispatch_dense(tmA, tmB, a, b_scale_mode == FP8Q_BSCALE_ROW1x128, true, tiles, nullptr, 0,
+  return dispatch_dense(tmA, tmB, tmA, a, b_scale_mode == FP8Q_BSCALE_ROW1x128, true, tiles, nullptr, 0,
                         static_cast<cudaStream_t>(stream));
 }
 
@@ -603,8 +623,12 @@ int fp8_gemm_grouped(const uint8_t* A, const float* sA, int64_t ld_sa, const uin
                         ((N + Cfg1::kN - 1) / Cfg1::kN);
   if (bound > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
   const auto s = static_cast<cudaStream_t>(stream);
-  if (out_dtype == FP8Q_OUT_BF16) return run_gemm<true, false, true, true>(tmA, tmB, a, bound, nullptr, 0, s);
-  return run_gemm<true, false, true, false>(tmA, tmB, a, bound, nullptr, 0, s);
+  if (out_dtype == FP8Q_OUT_BF16) {
+    CUtensorMap tmC;
+    if ((st = encode_output_bf16(&tmC, C, N, max_sum_M, N)) != FP8Q_OK) return st;
+    return run_gemm<true, false, true, true>(tmA, tmB, tmC, a, bound, nullptr, 0, s);
+  }
+  return run_gemm<true, false, true, false>(tmA, tmB, tmA, a, bound, nullptr, 0, s);
 }
 
 int fp8_gemm_nopromo(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB, float* C,
@@ -624,7 +648,7 @@ int fp8_gemm_nopromo(const uint8_t* A, const float* sA, const uint8_t* B, const 
   a.n_fastest = M > N;
   const int64_t tiles = dense_tiles(M, N);
   if (tiles > 0x7FFFFFFF) return FP8Q_ERR_SHAPE;
-  return run_gemm<false, false, false, false>(tmA, tmB, a, tiles, nullptr, 0,
+  return run_gemm<false, false, false, false>(tmA, tmB, tmA, a, tiles, nullptr, 0,
                                                      static_cast<cudaStream_t>(stream));
 }
 

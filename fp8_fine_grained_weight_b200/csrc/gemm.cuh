@@ -144,13 +144,16 @@ __device__ __forceinline__ Unit unit_at(int i, const GemmArgs& p, int unit0, int
 
 constexpr uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-template <bool ROW_B = false>
+// TSTORE: the tile's bf16 output leaves through shared memory and TMA stores (a 64 KB
+// staging area, one 8 KB slice per epilogue warp), so the epilogue warps go on to the next
+// tile while the stores drain; the operand ring then has 3 stages instead of 4.
+template <bool ROW_B = false, bool TSTORE = false>
 struct GemmCfg {
   static constexpr int kN = 256;                        // output columns per tile (MMA N)
   static constexpr int kTileM = 128;                    // output rows per tile (MMA M)
   static constexpr int kAccBufs = kTmemCols / kN;       // TMEM accumulators (groups in flight)
   static constexpr int kSetCols = kN / 2;               // columns per epilogue warpgroup
-  static constexpr int kStages = 4;
+  static constexpr int kStages = TSTORE ? 3 : 4;
   static constexpr int kBBox = kN;                      // B rows per TMA box
   static constexpr uint32_t kABytes = 128 * kBK;        // per stage
   static constexpr uint32_t kBBytes = kN * kBK;
@@ -164,7 +167,7 @@ struct GemmCfg {
   // in ROW mode; its kN / 128 block scales, padded to 4, otherwise).  One barrier wait
   // and one release per slot, not per group.
   static constexpr int kSlotGroups = 4;
-  static constexpr int kScaleSlots = ROW_B ? 4 : 6;
+  static constexpr int kScaleSlots = ROW_B ? 4 : (TSTORE ? 5 : 6);
   static constexpr uint32_t kGroupFloats = 128 + (ROW_B ? kN : 4);
   static constexpr uint32_t kSlotFloats = kSlotGroups * kGroupFloats;
   // full[S], empty[S], tfull[NB], tempty[NB], drain, sfull[R], sempty[R]
@@ -173,7 +176,10 @@ struct GemmCfg {
   static constexpr uint32_t sched = align_up(misc + 16, 16);          // int[kMaxGroups + 1]
   static constexpr uint32_t sbrow = align_up(sched + 4 * (kMaxGroups + 1), 128);  // float[2][2][128]
   static constexpr uint32_t sring = align_up(sbrow + 4 * 2 * 2 * 128, 128);  // float[R][kSlotFloats]
-  static constexpr uint32_t end = sring + 4 * kScaleSlots * kSlotFloats;
+  static constexpr uint32_t kStageWarpBytes = 32 * kSetCols * 2;     // 32 rows of bf16
+  static constexpr uint32_t stage = align_up(sring + 4 * kScaleSlots * kSlotFloats, 1024);
+  static constexpr uint32_t end = TSTORE ? stage + kEpiWarps * kStageWarpBytes
+                                         : sring + 4 * kScaleSlots * kSlotFloats;
   static constexpr uint32_t smem_bytes = end + 1024;                  // + base alignment slack
   static_assert(a % 1024 == 0 && b % 1024 == 0 && kABytes % 1024 == 0 && kBBytes % 1024 == 0,
                 "swizzle atoms");
@@ -182,7 +188,12 @@ struct GemmCfg {
   static_assert(kSetCols % 64 == 0 && kAccBufs >= 2, "64-column loads; two accumulators");
   static_assert(kN % 16 == 0 && kN <= 256 && kBBox <= 256, "MMA N and TMA box");
   static_assert(smem_bytes <= 232448, "fits the 227 KB opt-in shared memory");
+  static_assert(!TSTORE || (kSetCols == 128 && stage % 1024 == 0), "two 64-column swizzled boxes per warp");
 };
+
+// The configuration a promoted-GEMM instantiation runs with (host and device agree on it).
+template <bool PROMOTE, bool ROW_B, bool OUT_BF16, bool QOUT>
+using GemmCfgOf = GemmCfg<ROW_B, PROMOTE && !ROW_B && OUT_BF16 && !QOUT>;
 
 // Output tile of index t: first row of A, row bound for stores, first row of B (in the
 // stacked [E*N, K] weights), first output column, expert.
@@ -309,8 +320,10 @@ __device__ __forceinline__ void store_rows_by_quads(uint4 (&v)[NC], uint8_t* my_
 template <bool PROMOTE, bool ROW_B, bool GROUPED, bool OUT_BF16, bool QOUT = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_fp8_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA,
-                                const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
-  using Cfg = GemmCfg<ROW_B>;
+                                const __grid_constant__ CUtensorMap tmB,
+                                const __grid_constant__ CUtensorMap tmC, const GemmArgs p) {
+  using Cfg = GemmCfgOf<PROMOTE, ROW_B, OUT_BF16, QOUT>;
+  constexpr bool TSTORE = PROMOTE && !ROW_B && OUT_BF16 && !QOUT;
   constexpr int S = Cfg::kStages;
   constexpr int NB = Cfg::kAccBufs;
   constexpr int kN = Cfg::kN;
@@ -660,9 +673,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             hv[j].z = *reinterpret_cast<uint32_t*>(&h2);
             hv[j].w = *reinterpret_cast<uint32_t*>(&h3);
           }
-          if (p.C != nullptr)
+          if constexpr (TSTORE) {
+            // Rows of this warp all inside C's tile rows (always, dense: TMA drops rows past
+            // M): through this warp's staging slice and two TMA stores.  A warp whose rows
+            // cross an expert's end stores directly, masked by row.
+            if (tl.row0 + row_in_tile - lane + 32 <= tl.row_end || !GROUPED) {
+              const uint32_t stg = sbase + Cfg::stage + ew * Cfg::kStageWarpBytes;
+              if (lane == 0) bulk_wait_read_all();   // the previous tile's stores have read it
+              __syncwarp();
+              // two boxes of 64 columns x 32 rows, 128-byte rows, 128-byte swizzle: chunk c
+              // of row r at position c ^ (r % 8), so each quarter-warp covers all banks
+#pragma unroll
+              for (int j = 0; j < kSetCols / 8; ++j)
+                st_shared_v4(stg + (j >> 3) * 4096 + lane * 128 + (((j & 7) ^ (lane & 7)) << 4), hv[j]);
+              fence_proxy_async_shared();
+              __syncwarp();
+              if (lane == 0) {
+                const int32_t y = static_cast<int32_t>(tl.row0 + row_in_tile - lane);
+                tma_store_2d(&tmC, stg, static_cast<int32_t>(n0), y);
+                tma_store_2d(&tmC, stg + 4096, static_cast<int32_t>(n0 + 64), y);
+                bulk_commit_group();
+              }
+            } else {
+              store_rows_by_quads(hv, reinterpret_cast<uint8_t*>(reinterpret_cast<__nv_bfloat16*>(p.C) + m * p.ldc + n0),
+                                  row_ok);
+            }
+          } else if (p.C != nullptr) {
             store_rows_by_quads(hv, reinterpret_cast<uint8_t*>(reinterpret_cast<__nv_bfloat16*>(p.C) + m * p.ldc + n0),
                                 row_ok);
+          }
           if constexpr (QOUT) {
             // this thread's segment is exactly one 1x128 tile of the output row
             static_assert(kSetCols == 128 && !GROUPED, "one 1x128 output tile per epilogue thread");
@@ -699,6 +738,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 
   // ---------------------------------------------------------------- teardown
+  if (TSTORE && warp >= kEpiWarp0 && (threadIdx.x & 31) == 0) bulk_wait_all();   // stores done
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
