@@ -121,6 +121,8 @@ __device__ __forceinline__ uint2 quant8_with(const uint4& v, Q q) {
 }
 
 // Quantize NV vectors of 8 bf16 with one tile scale; the quotient rule is chosen once.
+// (All three rules inline: the 1x128 and 128x128 kernels measured slower with the rare
+// rules out of line, unlike the fused row + transposed kernel below.)
 template <int NV>
 __device__ __forceinline__ void quant_vectors(const uint4 (&v)[NV], const Quotient& qd, uint2 (&o)[NV]) {
   if (qd.mode == kExactRcp) {
@@ -302,6 +304,21 @@ struct PairGeneral {            // any rule, decided per call
     return NEG ? make_float2(q(-x.x), q(-x.y)) : make_float2(q(x.x), q(x.y));
   }
 };
+// The general rule out of line, for the fused row + transposed kernel: there only warps
+// whose tiles do not all share the usual rule take it, and inlining its division at
+// every call site multiplied the kernel's code size (83 KB against 21 KB).
+__device__ __noinline__ float2 pair_quotient_general(uint32_t w, float s, float r, int mode) {
+  Quotient q(s);
+  q.r = r;
+  q.mode = mode;
+  return make_float2(q(bf16lo(w)), q(bf16hi(w)));
+}
+struct PairGeneralCall {
+  float s, r;
+  int mode;
+  __device__ __forceinline__ explicit PairGeneralCall(const Quotient& q) : s(q.s), r(q.r), mode(q.mode) {}
+  __device__ __forceinline__ float2 operator()(uint32_t w) const { return pair_quotient_general(w, s, r, mode); }
+};
 
 // Runs body(pair quotient of the calling lane's tile) with the rule picked once per warp.
 template <bool NEG, typename Body>
@@ -309,6 +326,22 @@ __device__ __forceinline__ void with_pair_quotient(const Quotient& q, Body body)
   if (__all_sync(0xffffffffu, q.mode == kCorrected)) body(PairCorrected<NEG>(q));
   else if (__all_sync(0xffffffffu, q.mode == kExactRcp)) body(PairExact<NEG>(q));
   else body(PairGeneral<NEG>(q));
+}
+
+// The same with one specialised rule: the one a scale mode almost always gives (the exact
+// reciprocal for power-of-two scales, the corrected one for FP32 scales); any warp whose
+// tiles differ takes the general rule out of line.  Two copies of the body instead of
+// three, one of them small, keep the kernel's code small (instruction fetch was its
+// largest stall).
+template <bool POW2, typename Body>
+__device__ __forceinline__ void with_pair_quotient_for(const Quotient& q, Body body) {
+  constexpr bool NEG = !POW2;
+  if (__all_sync(0xffffffffu, q.mode == (POW2 ? kExactRcp : kCorrected))) {
+    if constexpr (POW2) body(PairExact<NEG>(q));
+    else body(PairCorrected<NEG>(q));
+  } else {
+    body(PairGeneralCall(q));
+  }
 }
 
 // In-quad 4x4 transpose of 32-bit words: lane q of a group of 4 lanes holds row q of a
@@ -368,7 +401,7 @@ __global__ void __launch_bounds__(256, 6) quant_act_dual_kernel(const __grid_con
   if (!__syncthreads_and(mbar_wait(bar, 0, kSiteDual, nullptr))) return;
 
   // ---- rows: lane l4 of the team of row r holds chunks (l4 + 4 j + 4 (r & 1)) % 16
-#pragma unroll
+#pragma unroll 1
   for (int pass = 0; pass < 2; ++pass) {
     const uint32_t r = warp * 16 + pass * 8 + (lane >> 2);  // row inside the tile
     const int64_t m = m0 + r;
@@ -386,7 +419,7 @@ __global__ void __launch_bounds__(256, 6) quant_act_dual_kernel(const __grid_con
     a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
     const float sc = tile_scale(a, POW2);
     uint8_t* dst = q + m * ldq + k0;
-    with_pair_quotient<!POW2>(Quotient(sc), [&](const auto& qd) {
+    with_pair_quotient_for<POW2>(Quotient(sc), [&](const auto& qd) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const uint4 w = v[j];
@@ -405,7 +438,7 @@ __global__ void __launch_bounds__(256, 6) quant_act_dual_kernel(const __grid_con
 
   // ---- columns 16 warp + 8 h + lane / 4 (h = 0, 1), all 128 rows
   const int quad = lane >> 2;                  // column inside the 8-column block
-#pragma unroll
+#pragma unroll 1
   for (int h = 0; h < 2; ++h) {
     const uint32_t chunk = static_cast<uint32_t>(2 * warp + h);    // 16-byte chunk of the rows
     // lane l addresses row 8 (rb4 + l / 8) + l % 8 of 4 consecutive 8-row blocks
@@ -424,7 +457,7 @@ __global__ void __launch_bounds__(256, 6) quant_act_dual_kernel(const __grid_con
     const float sc = tile_scale(a, POW2);
     // pairs of codes: rows 8b + 2 l4 (low byte) and 8b + 2 l4 + 1
     uint32_t vv[8];                            // vv[c]: rows 16c + 2 l4, +1 | 16c + 8 + 2 l4, +1
-    with_pair_quotient<!POW2>(Quotient(sc), [&](const auto& qd) {
+    with_pair_quotient_for<POW2>(Quotient(sc), [&](const auto& qd) {
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const float2 e0 = qd(w2[2 * c]);
