@@ -204,12 +204,16 @@ def run_gpu(args, rank, world):
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device()) as clk:
+
+    def enqueue_steps():
         for i in range(args.steps):
             flush_l2()             # outside the step's events
-            torch.cuda._sleep(200_000)   # the host enqueues the step before the GPU reaches it
             step(evs[i])
-        torch.cuda.synchronize()
+
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        # every step is enqueued behind a spin that outlasts the enqueueing, so the GPU runs
+        # the steps back to back and no host latency falls inside a step's events
+        _enqueue_ahead(enqueue_steps, lead_ms=max(20.0, 0.6 * args.steps))
     barrier(world)
     t_act = [e[0].elapsed_time(e[1]) for e in evs]
     t_w = [e[1].elapsed_time(e[2]) for e in evs]
@@ -332,27 +336,50 @@ def _spread(ts) -> dict:
             "best": round(min(ts), 5)}
 
 
+def _enqueue_ahead(enqueue, lead_ms=20.0, max_ms=4000.0):
+    """Runs enqueue() -- which only enqueues GPU work (and timing events) on the current
+    stream -- behind a spin kernel on that stream that outlasts the host's enqueueing, so
+    that the GPU never waits for the host between the enqueued events: host-side latency (a
+    busy host, Python argument checks) cannot show up inside a timed region.  If the spin
+    ended before the host finished enqueueing, the work is run again behind a spin twice as
+    long.  Returns enqueue()'s result once its work has completed."""
+    import torch
+    stream = torch.cuda.current_stream()
+    while True:
+        torch.cuda.synchronize()
+        torch.cuda._sleep(int(lead_ms * 2.0e6))    # ~lead_ms at 2 GHz (longer at lower clocks)
+        lead_end = torch.cuda.Event()
+        lead_end.record(stream)
+        out = enqueue()
+        caught_up = lead_end.query()
+        torch.cuda.synchronize()
+        if not caught_up or lead_ms >= max_ms:
+            return out
+        lead_ms *= 2
+
+
 def _time_ms(fn, reps, flush_l2, warmup=2):
     """Mean device time of fn() over reps, L2 flushed before each (outside the events).
     Untimed warm-up calls first: a kernel variant's first launch pays one-time setup.
-    All reps are enqueued before the host waits, and after each flush the GPU spins for
-    ~0.1 ms, so the host stays ahead of the GPU: host-side latency (a busy host, Python
-    argument checks) never shows up as idle time between a rep's events."""
+    All reps are enqueued behind a spin that outlasts the enqueueing (_enqueue_ahead)."""
     import torch
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
-    evs = []
-    for _ in range(reps):
-        flush_l2()
-        torch.cuda._sleep(200_000)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        fn()
-        e1.record(stream)
-        evs.append((e0, e1))
-    torch.cuda.synchronize()
+
+    def enqueue():
+        evs = []
+        for _ in range(reps):
+            flush_l2()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            evs.append((e0, e1))
+        return evs
+
+    evs = _enqueue_ahead(enqueue, lead_ms=max(20.0, 1.0 * reps))
     return sum(e0.elapsed_time(e1) for e0, e1 in evs) / reps
 
 
