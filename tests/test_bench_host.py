@@ -1,5 +1,6 @@
 """Host-side logic of bench.py, without a GPU: the max over ranks on two gloo ranks, the
-dense step's GEMM choice, and the reference arm's JSON line."""
+dense step's GEMM choice, the reference arm's JSON line, and the timing loop's rule for
+keeping the host ahead of the GPU (_enqueue_ahead, against a stand-in for torch.cuda)."""
 import json
 import os
 import socket
@@ -185,3 +186,61 @@ def test_reference_arm_line_on_rank0_and_silence_elsewhere():
     r1 = _run_bench("--impl", "reference", "--steps", "1", "--warmup", "1", "--workload", "tiny",
                     env={"RANK": "1", "WORLD_SIZE": "2"})
     assert r1.returncode == 0 and r1.stdout.strip() == ""
+
+
+class _FakeCuda:
+    """Stand-in for torch.cuda in _enqueue_ahead: records the spin lengths and answers the
+    spin's completion query from a script (True: the spin had ended before the host
+    finished enqueueing)."""
+
+    def __init__(self, caught_up):
+        self.caught_up = list(caught_up)
+        self.spins = []
+        self.syncs = 0
+        fake = self
+
+        class Event:
+            def record(self, stream):
+                pass
+
+            def query(self):
+                return fake.caught_up.pop(0)
+
+        self.Event = Event
+
+    def current_stream(self):
+        return object()
+
+    def synchronize(self):
+        self.syncs += 1
+
+    def _sleep(self, cycles):
+        self.spins.append(cycles)
+
+
+def _run_enqueue_ahead(monkeypatch, caught_up, **kw):
+    import torch
+    fake = _FakeCuda(caught_up)
+    for name in ("Event", "current_stream", "synchronize", "_sleep"):
+        monkeypatch.setattr(torch.cuda, name, getattr(fake, name))
+    calls = []
+    out = bench._enqueue_ahead(lambda: calls.append(len(calls)) or len(calls), **kw)
+    return fake, calls, out
+
+
+def test_enqueue_ahead_keeps_the_first_run_when_the_spin_outlasted_the_host(monkeypatch):
+    fake, calls, out = _run_enqueue_ahead(monkeypatch, [False], lead_ms=20.0)
+    assert calls == [0] and out == 1
+    assert fake.spins == [int(20.0 * 2.0e6)]
+    assert fake.syncs == 2          # before the spin, and after the work before returning
+
+
+def test_enqueue_ahead_doubles_the_spin_until_it_outlasts_the_host(monkeypatch):
+    fake, calls, out = _run_enqueue_ahead(monkeypatch, [True, True, False], lead_ms=20.0)
+    assert calls == [0, 1, 2] and out == 3      # the work of the last run is returned
+    assert fake.spins == [int(ms * 2.0e6) for ms in (20.0, 40.0, 80.0)]
+
+
+def test_enqueue_ahead_stops_at_its_longest_spin(monkeypatch):
+    fake, calls, out = _run_enqueue_ahead(monkeypatch, [True] * 10, lead_ms=20.0, max_ms=80.0)
+    assert len(calls) == 3 and fake.spins == [int(ms * 2.0e6) for ms in (20.0, 40.0, 80.0)]
