@@ -14,30 +14,33 @@
 //
 // Roles (384-thread CTAs, one per SM, persistent over 128 x 256 output tiles):
 //   warp 0      TMA producer: per K-group, the A tile [128 rows x 128 B] and the B tile
-//               [256 rows x 128 B] into a 4-stage shared-memory ring (128-byte swizzle).
+//               [256 rows x 128 B] into a shared-memory ring (128-byte swizzle; 4 stages,
+//               3 where the bf16 output is staged for TMA stores).
 //   warp 1      TMEM owner and MMA issuer: per group 4 x tcgen05.mma kind::f8f6f4 (M128
 //               N256 K32) into a fresh 256-column TMEM accumulator (two, alternating),
-//               then tcgen05.commit to free the smem stage and to publish the partial.
-//               It waits for the stage's operands before the accumulator: the operands
-//               are normally in place long before, while the accumulator comes free just
-//               in time, and the MMAs should follow its release with nothing in between.
+//               then one tcgen05.commit on the stage's barrier, which both frees the smem
+//               stage and publishes the partial to the epilogue.  It waits for the
+//               stage's operands before the accumulator: the operands are normally in
+//               place long before, while the accumulator comes free just in time, and
+//               the MMAs should follow its release with nothing in between.
 //   warp 2      scale producer: for every group, ahead of the epilogue, copies the
 //               tile's 128 row scales of A and its B scales (2 block scales, or 256
-//               column scales) into a shared-memory ring with cp.async.  The small copies
-//               queue behind the operand stream in L2, so the ring is deep (24 groups for
-//               block scales, 16 for column scales).
+//               column scales) into a shared-memory ring of four-group slots with
+//               cp.async (20-24 groups ahead for block scales, 16 for column scales).
 //   warp 3      idle (it completes the first warpgroup).
 //   warps 4-11  promotion/epilogue: warp w reads TMEM lanes 32*(w%4).. and the tile's
 //               columns 128*((w-4)/4)..; per group two 64-column tcgen05.ld and
 //               acc += P * scale in FP32 registers (f32x2 FMAs); the accumulator is freed
-//               after the second load; at the end of the tile: convert and store C.
+//               after the second load; at the end of the tile: convert and store C (bf16
+//               with block scales: through a per-warp shared-memory slice and TMA stores).
 //
 // Measured on B200 and not kept (same operands, same parity): a CTA pair with 256 x 256
 // tiles (a third less L2 traffic per FLOP, but the cross-CTA accumulator release slowed
-// every group); MMAs issued as two N = 128 halves into four TMEM slices (more slack per
-// slice, but a single issuing thread then cannot keep the tensor pipe fed); 32-column
-// TMEM loads pipelined with the FMAs, within a group and across groups (the extra
-// registers spill).
+// every group); MMAs issued as two N = 128 halves into four TMEM slices, and 128 x 128
+// tiles with four accumulators (more slack per accumulator, but more operand traffic and
+// twice the per-group synchronisation); 32-column TMEM loads pipelined with the FMAs
+// (the extra registers spill); releases as one arrival per warp; block scales loaded by
+// the epilogue itself instead of the scale ring.
 //
 // Registers: the launch gives 168 per thread (3 warps per SM sub-partition).  The
 // first warpgroup gives registers back (setmaxnreg 40) and the two epilogue
